@@ -1,0 +1,314 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself.
+
+Each pin takes an oracle module ``o`` and raises AssertionError when the
+oracle disagrees with a closed form, an invariant, a brute-force computation
+on tiny inputs, or a value printed on the KVzip pages.  The same pins run
+against deliberately broken copies of the oracle (tests/test_oracle_pins.py)
+to show that each plausible mistake is caught by at least one of them.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _inputs(seed, B, G, n_in, n_c, d, chunks=1):
+    r = _rng(seed)
+    k_ctx = r.standard_normal((B, n_c, d))
+    qs = [r.standard_normal((B, G, n_in, d)) for _ in range(chunks)]
+    kss = [r.standard_normal((B, n_in, d)) for _ in range(chunks)]
+    return qs, kss, k_ctx
+
+
+# ---------------------------------------------------------------- scoring pins
+
+def pin_row_sums_and_range(o):
+    """Softmax rows sum to 1 (1e-12) and every score lies in (0, 1]."""
+    qs, kss, k_ctx = _inputs(1, 2, 3, 9, 20, 8, chunks=2)
+    scale = 1 / math.sqrt(8)
+    for q, ks in zip(qs, kss):
+        for b in range(2):
+            p = o.softmax_rows(o.chunk_logits(q[b], k_ctx[b], ks[b], scale))
+            assert np.allclose(p.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+    S = o.score_context(qs, kss, k_ctx)
+    assert np.all(S > 0) and np.all(S <= 1.0 + 1e-15)
+
+
+def pin_uniform_queries(o):
+    """Q = 0: row (g, i) is uniform over n_c + i + 1 keys, so S[j] = 1/(n_c + 1)
+    (the row i = 0 wins) and lse_i = log(n_c + i + 1)."""
+    for (G, n_in, n_c, d, chunks) in [(1, 5, 7, 4, 1), (3, 6, 11, 8, 2), (2, 17, 33, 16, 3)]:
+        r = _rng(2)
+        k_ctx = r.standard_normal((1, n_c, d)) * 3
+        qs = [np.zeros((1, G, n_in, d)) for _ in range(chunks)]
+        kss = [r.standard_normal((1, n_in, d)) for _ in range(chunks)]
+        S = o.score_context(qs, kss, k_ctx)
+        assert np.allclose(S, 1.0 / (n_c + 1), rtol=1e-13, atol=0)
+        _, lse = o.unit_chunk_scores(qs[0][0], k_ctx[0], kss[0][0])
+        i = np.tile(np.arange(n_in), G)
+        assert np.allclose(lse, np.log(n_c + i + 1), rtol=1e-13, atol=1e-13)
+
+
+def pin_logistic(o):
+    """n_c = 1, n_in = 1, G = 1: S = sigmoid(s - s') with s = q.k / sqrt(d),
+    s' = q.k_self / sqrt(d) (the single row sees one context key and itself)."""
+    r = _rng(3)
+    for d in (4, 64, 128):
+        for _ in range(5):
+            q = r.standard_normal((1, 1, 1, d))
+            k = r.standard_normal((1, 1, d))
+            ks = r.standard_normal((1, 1, d))
+            s = float(q[0, 0, 0] @ k[0, 0]) / math.sqrt(d)
+            sp = float(q[0, 0, 0] @ ks[0, 0]) / math.sqrt(d)
+            S = o.score_context([q], [ks], k)
+            want = 1.0 / (1.0 + math.exp(sp - s))
+            assert abs(S[0, 0] - want) <= 1e-14, (S[0, 0], want)
+
+
+def pin_dominant_key(o):
+    """A context key far larger than the rest and aligned with one query row
+    takes essentially all of that row's mass: S -> 1 for that key, while a
+    mean over rows would stay near 1/rows."""
+    r = _rng(4)
+    G, n_in, n_c, d = 2, 8, 30, 16
+    q = r.standard_normal((1, G, n_in, d))
+    k = r.standard_normal((1, n_c, d))
+    ks = r.standard_normal((1, n_in, d))
+    u = q[0, 1, 5] / np.linalg.norm(q[0, 1, 5])
+    k[0, 17] = 400.0 * u
+    S = o.score_context([q], [ks], k)
+    assert S[0, 17] > 1 - 1e-12, S[0, 17]
+
+
+def _bruteforce_pure_python(qs, kss, k_ctx, scale):
+    """Dense, unchunked: every row of every chunk in one matrix whose columns
+    are the n_c context keys followed by the self keys of *all* chunks; a row
+    of chunk c at position i sees context keys and chunk c's self keys 0..i
+    (block-diagonal causal mask).  Global column max over all rows."""
+    B, n_c, d = k_ctx.shape
+    out = [[0.0] * n_c for _ in range(B)]
+    for b in range(B):
+        cols = [list(map(float, k_ctx[b, j])) for j in range(n_c)]
+        owner = [(-1, j) for j in range(n_c)]
+        for c, ks in enumerate(kss):
+            for jp in range(ks.shape[1]):
+                cols.append(list(map(float, ks[b, jp])))
+                owner.append((c, jp))
+        for c, q in enumerate(qs):
+            G, n_in = q.shape[1], q.shape[2]
+            for g in range(G):
+                for i in range(n_in):
+                    row = list(map(float, q[b, g, i]))
+                    logit = []
+                    for col, (oc, jp) in zip(cols, owner):
+                        visible = oc == -1 or (oc == c and jp <= i)
+                        if visible:
+                            logit.append(scale * sum(x * y for x, y in zip(row, col)))
+                        else:
+                            logit.append(None)
+                    mx = max(v for v in logit if v is not None)
+                    z = sum(math.exp(v - mx) for v in logit if v is not None)
+                    for j in range(n_c):
+                        p = math.exp(logit[j] - mx) / z
+                        if p > out[b][j]:
+                            out[b][j] = p
+    return np.array(out)
+
+
+def pin_bruteforce_unchunked(o):
+    """Chunked running max == one dense unchunked matrix over all chunks' rows
+    with a block-diagonal causal self mask, on tiny inputs (pure Python)."""
+    cases = [  # (G, n_in, n_c, d, chunks)
+        (1, 8, 24, 4, 3),
+        (2, 11, 16, 16, 2),
+        (4, 6, 20, 8, 2),
+        (2, 19, 40, 128, 2),
+    ]
+    for seed, (G, n_in, n_c, d, chunks) in enumerate(cases):
+        qs, kss, k_ctx = _inputs(10 + seed, 2, G, n_in, n_c, d, chunks)
+        k_ctx[:, :3] *= 3.0
+        want = _bruteforce_pure_python(qs, kss, k_ctx, 1 / math.sqrt(d))
+        got = o.score_context(qs, kss, k_ctx)
+        assert np.allclose(got, want, rtol=1e-12, atol=0), np.abs(got / want - 1).max()
+
+
+def pin_invariants(o):
+    """Chunk order, query-head order and duplicated query heads leave S
+    unchanged; permuting the context keys permutes S; re-scoring a chunk is
+    idempotent."""
+    qs, kss, k_ctx = _inputs(20, 2, 3, 10, 25, 8, chunks=3)
+    S = o.score_context(qs, kss, k_ctx)
+    # chunk order
+    S2 = o.score_context(qs[::-1], kss[::-1], k_ctx)
+    assert np.array_equal(S, S2)
+    # query-head permutation and duplication
+    perm = [2, 0, 1]
+    S3 = o.score_context([q[:, perm] for q in qs], kss, k_ctx)
+    assert np.allclose(S, S3, rtol=1e-14, atol=0)
+    S4 = o.score_context([np.concatenate([q, q[:, :1]], axis=1) for q in qs], kss, k_ctx)
+    assert np.allclose(S, S4, rtol=1e-14, atol=0)
+    # key permutation
+    pk = _rng(21).permutation(25)
+    S5 = o.score_context(qs, kss, k_ctx[:, pk])
+    assert np.allclose(S5, S[:, pk], rtol=1e-13, atol=0)
+    # idempotent re-scoring
+    S6 = S.copy()
+    o.score_chunk(qs[1], k_ctx, kss[1], S6)
+    assert np.array_equal(S6, S)
+
+
+def pin_rows_see_own_prefix(o):
+    """Changing a self key j' changes only rows i >= j': checked through the
+    lse of each row (rows i < j' keep their lse exactly)."""
+    r = _rng(30)
+    G, n_in, n_c, d = 2, 9, 12, 8
+    q = r.standard_normal((G, n_in, d))
+    k = r.standard_normal((n_c, d))
+    ks = r.standard_normal((n_in, d))
+    _, lse0 = o.unit_chunk_scores(q, k, ks)
+    jp = 4
+    ks2 = ks.copy()
+    ks2[jp] += 5.0
+    _, lse1 = o.unit_chunk_scores(q, k, ks2)
+    i = np.tile(np.arange(n_in), G)
+    assert np.array_equal(lse0[i < jp], lse1[i < jp])
+    assert np.all(lse0[i >= jp] != lse1[i >= jp])
+
+
+# -------------------------------------------------------------- selection pins
+
+def pin_keep_count(o):
+    """k = ceil(r N): equals the exact decimal product for the workloads'
+    ratios and sizes (e.g. r = 0.3 of 2048 keys keeps 615)."""
+    cases = [(0.3, 2048), (0.3, 4194304), (0.3, 33554432), (0.5, 33554432),
+             (0.25, 47185920), (0.3, 66846720), (0.0, 100), (1.0, 100), (0.7, 10)]
+    for r, N in cases:
+        exact = Fraction(str(r)) * N
+        want = math.ceil(exact)
+        assert o.keep_count(r, N) == want, (r, N, o.keep_count(r, N), want)
+    assert o.keep_count(0.3, 2048) == 615
+
+
+def _check_selection(s, k, n_heads, keep, offsets, threshold):
+    s = np.asarray(s).reshape(-1)
+    N = s.size
+    kept = np.nonzero(keep)[0]
+    dropped = np.nonzero(keep == 0)[0]
+    assert kept.size == k
+    if k and dropped.size:
+        # every kept score is >= every dropped score
+        assert s[kept].min() >= s[dropped].max()
+        # ties at the boundary: kept ones have lower flat index than dropped ones
+        tau = s[kept].min()
+        tk = kept[s[kept] == tau]
+        td = dropped[s[dropped] == tau]
+        if td.size:
+            assert tk.max() < td.min()
+    if k:
+        assert threshold == s[kept].min()
+    else:
+        assert threshold == math.inf
+    cnt = keep.reshape(n_heads, -1).sum(axis=1)
+    assert offsets[0] == 0 and np.array_equal(np.diff(offsets), cnt)
+    assert offsets[-1] == k
+
+
+def pin_select_properties(o):
+    """The kept set is the unique set of size k with every kept score >= every
+    dropped one and ties kept lowest-index first; offsets are the exclusive
+    scan of per-head counts.  Random and tie-heavy arrays, r in {0, .3, .5, 1}."""
+    r = _rng(40)
+    for levels in (0, 8, 2, 1):
+        for n_heads, n_c in [(4, 50), (7, 33), (1, 200)]:
+            s = r.random((n_heads, n_c)) ** 4
+            if levels:
+                s = (np.floor(s * levels) + 1) / levels
+            s = s.astype(np.float32)
+            for frac in (0.0, 0.3, 0.5, 1.0):
+                k = o.keep_count(frac, s.size)
+                keep, offsets, thr = o.select(s.reshape(-1), k, n_heads)
+                _check_selection(s, k, n_heads, keep, offsets, thr)
+    keep, offsets, _ = o.select(np.ones(12, np.float32), 12, 3)
+    assert keep.all()
+
+
+def pin_select_bruteforce(o):
+    """Tiny arrays: the kept set equals the best-of-all-subsets answer under the
+    order (higher score, then lower index) found by exhaustive search."""
+    from itertools import combinations
+    r = _rng(41)
+    for trial in range(6):
+        n_heads, n_c = 2, 4
+        code = np.floor(r.random(n_heads * n_c) * 3).astype(np.int64)   # 0, 1, 2
+        s = (code / 3).astype(np.float32)
+        for k in range(0, 9):
+            best = None
+            for sub in combinations(range(8), k):
+                # preference: larger total score first (exact, in integer codes),
+                # then the lexicographically smaller sorted index list
+                key = (sum(int(code[i]) for i in sub), tuple(-i for i in sorted(sub)))
+                if best is None or key > best[0]:
+                    best = (key, sub)
+            keep, _, _ = o.select(s, k, n_heads)
+            assert set(np.nonzero(keep)[0].tolist()) == set(best[1]), (s, k)
+
+
+# ------------------------------------------------------------- compaction pins
+
+def pin_compact(o):
+    """Compacted rows equal the source rows byte for byte; positions ascend in
+    each head; kept bytes = k * d * 2 (bf16) * 2 (K and V)."""
+    r = _rng(50)
+    n_heads, n_c, d = 5, 37, 8
+    k = r.integers(0, 2**16, size=(n_heads, n_c, d), dtype=np.uint16)  # bf16 bit patterns
+    v = r.integers(0, 2**16, size=(n_heads, n_c, d), dtype=np.uint16)
+    s = r.random(n_heads * n_c).astype(np.float32)
+    kk = o.keep_count(0.4, s.size)
+    keep, offsets, _ = o.select(s, kk, n_heads)
+    ko, vo, pos = o.compact(k, v, keep, offsets)
+    assert ko.nbytes + vo.nbytes == kk * d * 2 * 2
+    for h in range(n_heads):
+        seg = pos[offsets[h]:offsets[h + 1]]
+        assert np.all(np.diff(seg) > 0)
+        assert np.array_equal(seg, np.nonzero(keep.reshape(n_heads, n_c)[h])[0])
+        assert np.array_equal(ko[offsets[h]:offsets[h + 1]], k[h, seg])
+        assert np.array_equal(vo[offsets[h]:offsets[h + 1]], v[h, seg])
+
+
+def pin_kv_size_table(o):
+    """The rebuttal's decoding table: KV cache size is linear in the kept ratio
+    (32.7 GB at ratio 1 -> 26.2, 19.6, 13.1, 6.5).  Compaction bytes from the
+    oracle, scaled to 32.7 GB at ratio 1, reproduce every printed size to the
+    printed 0.1 GB."""
+    with open(os.path.join(GOLDEN, "kv_size_vs_ratio.json")) as f:
+        g = json.load(f)
+    r = _rng(51)
+    n_heads, n_c, d = 8, 1000, 4
+    s = r.random(n_heads * n_c).astype(np.float32)
+    k = np.zeros((n_heads, n_c, d), np.uint16)
+    full = None
+    for ratio, gb in zip(g["ratio"], g["kv_cache_gb"]):
+        kk = o.keep_count(ratio, s.size)
+        keep, offsets, _ = o.select(s, kk, n_heads)
+        ko, vo, _ = o.compact(k, k, keep, offsets)
+        nbytes = ko.nbytes + vo.nbytes
+        if full is None:
+            full = nbytes
+        assert round(32.7 * nbytes / full, 1) == gb, (ratio, 32.7 * nbytes / full, gb)
+
+
+SCORING_PINS = [pin_row_sums_and_range, pin_uniform_queries, pin_logistic, pin_dominant_key,
+                pin_bruteforce_unchunked, pin_invariants, pin_rows_see_own_prefix]
+SELECT_PINS = [pin_keep_count, pin_select_properties, pin_select_bruteforce]
+COMPACT_PINS = [pin_compact, pin_kv_size_table]
+ALL_PINS = SCORING_PINS + SELECT_PINS + COMPACT_PINS

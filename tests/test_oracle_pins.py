@@ -1,0 +1,163 @@
+"""The CPU oracle against its pins, and planted mistakes against the same pins.
+
+A planted mistake lives in a private copy of the oracle module loaded for the
+test; the real oracle is never modified.
+"""
+import importlib.util
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from tests import oracle_pins as P
+
+ORACLE_FILE = os.path.join(os.path.dirname(os.path.dirname(__file__)), "oracle", "kvzip_oracle.py")
+
+
+@pytest.mark.parametrize("pin", P.ALL_PINS, ids=lambda f: f.__name__)
+def test_oracle_pin(pin):
+    pin(oracle)
+
+
+def _fresh_copy():
+    spec = importlib.util.spec_from_file_location("kvzip_oracle_mutant", ORACLE_FILE)
+    m = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(m)
+    return m
+
+
+def _mut_drop_diagonal(m):
+    def mask(G, n_in):
+        i = np.tile(np.arange(n_in), G)
+        return np.arange(n_in)[None, :] < i[:, None]
+    m.causal_self_mask = mask
+
+
+def _mut_anticausal(m):
+    def mask(G, n_in):
+        i = np.tile(np.arange(n_in), G)
+        return np.arange(n_in)[None, :] >= i[:, None]
+    m.causal_self_mask = mask
+
+
+def _mut_row_order(m):
+    # rows taken i-major instead of g-major: the row -> position map is wrong
+    def mask(G, n_in):
+        i = np.repeat(np.arange(n_in), G)
+        return np.arange(n_in)[None, :] <= i[:, None]
+    m.causal_self_mask = mask
+
+
+def _mut_no_self_in_normaliser(m):
+    orig = m.chunk_logits
+
+    def logits(q, k_ctx, k_self, scale):
+        a = orig(q, k_ctx, k_self, scale)
+        a[:, k_ctx.shape[0]:] = -np.inf
+        return a
+    m.chunk_logits = logits
+
+
+def _mut_no_scale(m):
+    orig = m.chunk_logits
+    m.chunk_logits = lambda q, k, ks, scale: orig(q, k, ks, 1.0)
+
+
+def _mut_mean(m):
+    def ucs(q, k_ctx, k_self, scale=None):
+        k_ctx = np.asarray(k_ctx, np.float64)
+        if scale is None:
+            scale = 1 / math.sqrt(k_ctx.shape[1])
+        a = m.chunk_logits(q, k_ctx, k_self, scale)
+        p = m.softmax_rows(a)
+        mx = a.max(axis=1)
+        return p[:, :k_ctx.shape[0]].mean(axis=0), mx + np.log(np.exp(a - mx[:, None]).sum(1))
+    m.unit_chunk_scores = ucs
+
+
+def _mut_sum_over_chunks(m):
+    def score_chunk(q, k_ctx, k_self, scores, scale=None):
+        for b in range(len(q)):
+            s_c, _ = m.unit_chunk_scores(q[b], k_ctx[b], k_self[b], scale)
+            scores[b] += s_c
+        return scores
+    m.score_chunk = score_chunk
+
+
+def _mut_transposed_keys(m):
+    orig = m.chunk_logits
+
+    def logits(q, k_ctx, k_self, scale):
+        q = np.asarray(q, np.float64)
+        # uses the self keys of the wrong end of the chunk (reversed order)
+        return orig(q, k_ctx, np.asarray(k_self)[::-1], scale)
+    m.chunk_logits = logits
+
+
+def _mut_floor_count(m):
+    m.keep_count = lambda r, N: int(math.floor(r * N))
+
+
+def _mut_tie_high_index(m):
+    orig = m.select
+
+    def select(scores, k, n_heads):
+        s = np.asarray(scores).reshape(-1)
+        N = s.size
+        order = np.lexsort((-np.arange(N), -s.astype(np.float64)))
+        keep = np.zeros(N, np.uint8)
+        keep[order[:k]] = 1
+        cnt = keep.reshape(n_heads, -1).sum(1)
+        off = np.concatenate([[0], np.cumsum(cnt)]).astype(np.int64)
+        return keep, off, (float(s[order[k - 1]]) if k else math.inf)
+    m.select = select
+
+
+def _mut_uniform_head_budget(m):
+    def select(scores, k, n_heads):
+        s = np.asarray(scores).reshape(n_heads, -1)
+        keep = np.zeros_like(s, dtype=np.uint8)
+        per = k // n_heads
+        for h in range(n_heads):
+            keep[h, np.argsort(-s[h], kind="stable")[:per]] = 1
+        keep = keep.reshape(-1)
+        cnt = keep.reshape(n_heads, -1).sum(1)
+        off = np.concatenate([[0], np.cumsum(cnt)]).astype(np.int64)
+        kept = s.reshape(-1)[keep == 1]
+        return keep, off, (float(kept.min()) if kept.size else math.inf)
+    m.select = select
+
+
+def _mut_positions_descending(m):
+    orig = m.compact
+
+    def compact(k, v, keep, offsets):
+        ko, vo, pos = orig(k, v, keep, offsets)
+        for h in range(len(offsets) - 1):
+            a, b = int(offsets[h]), int(offsets[h + 1])
+            ko[a:b], vo[a:b], pos[a:b] = ko[a:b][::-1].copy(), vo[a:b][::-1].copy(), pos[a:b][::-1].copy()
+        return ko, vo, pos
+    m.compact = compact
+
+
+MUTANTS = [_mut_drop_diagonal, _mut_anticausal, _mut_row_order, _mut_no_self_in_normaliser,
+           _mut_no_scale, _mut_mean, _mut_sum_over_chunks, _mut_transposed_keys,
+           _mut_floor_count, _mut_tie_high_index, _mut_uniform_head_budget,
+           _mut_positions_descending]
+
+
+@pytest.mark.parametrize("mutate", MUTANTS, ids=lambda f: f.__name__)
+def test_planted_mistake_is_caught(mutate):
+    m = _fresh_copy()
+    mutate(m)
+    caught = []
+    for pin in P.ALL_PINS:
+        try:
+            pin(m)
+        except AssertionError:
+            caught.append(pin.__name__)
+        except (ValueError, IndexError, ZeroDivisionError, FloatingPointError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught {mutate.__name__}"
