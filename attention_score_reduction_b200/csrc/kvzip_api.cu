@@ -1,0 +1,218 @@
+// Host side of the libkvzip C ABI (declared in include/kvzip.h): argument
+// validation, workspace carving and kernel launches.  No allocation, no
+// synchronisation (except kvzip_workspace_status), no CPU compute path.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <climits>
+#include <cmath>
+#include <cstdint>
+
+#include "kvzip.h"
+#include "kvzip_internal.h"
+
+namespace {
+
+std::atomic<uint64_t> g_timeout_ns{2000000000ull};
+std::atomic<int> g_last_launches{0};
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int64_t row_pad(int64_t R) { return (R + kvzip::kRowPad - 1) / kvzip::kRowPad * kvzip::kRowPad; }
+
+kvzip_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KVZIP_OK : KVZIP_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* kvzip_status_string(kvzip_status s) {
+  switch (s) {
+    case KVZIP_OK: return "ok";
+    case KVZIP_ERR_INVALID_ARG: return "invalid argument";
+    case KVZIP_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case KVZIP_ERR_CUDA: return "CUDA error";
+    case KVZIP_ERR_TIMEOUT: return "kernel pipeline wait timed out";
+  }
+  return "unknown status";
+}
+
+void kvzip_set_wait_timeout_ns(uint64_t ns) {
+  g_timeout_ns.store(ns == 0 ? 2000000000ull : ns);
+}
+
+/* Number of kernel launches the most recent successful call enqueued (testing aid). */
+int kvzip_last_launch_count(void) { return g_last_launches.load(); }
+
+size_t kvzip_score_workspace_size(int B, int G, int n_in) {
+  if (B < 0 || G < 0 || n_in < 0) return 0;
+  const int64_t R = static_cast<int64_t>(G) * n_in;
+  return kvzip::kScoreWsHeader + static_cast<size_t>(B) * static_cast<size_t>(row_pad(R)) * 4;
+}
+
+static kvzip_status score_passes(int passes, kvzip_dtype dt, const void* q, const void* k_ctx,
+                                 const void* k_self, float* scores, int B, int G, int n_in,
+                                 int n_c, int d, float scale, void* workspace, size_t ws_bytes,
+                                 void* stream) {
+  if (dt != KVZIP_BF16 && dt != KVZIP_F32) return KVZIP_ERR_INVALID_ARG;
+  if (B < 0 || G < 0 || n_in < 0 || n_c < 0) return KVZIP_ERR_INVALID_ARG;
+  if (d != 128 && d != 256) return d > 0 ? KVZIP_ERR_UNSUPPORTED : KVZIP_ERR_INVALID_ARG;
+  if (B == 0 || G == 0 || n_in == 0 || n_c == 0) return KVZIP_OK;
+  if (!q || !k_ctx || !k_self || !scores || !workspace) return KVZIP_ERR_INVALID_ARG;
+  const int64_t R = static_cast<int64_t>(G) * n_in;
+  if (R > INT_MAX - kvzip::kRowPad || B > 65535) return KVZIP_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k_ctx, 16) || !aligned(k_self, 16) || !aligned(scores, 4) ||
+      !aligned(workspace, 256))
+    return KVZIP_ERR_INVALID_ARG;
+  if (ws_bytes < kvzip_score_workspace_size(B, G, n_in)) return KVZIP_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || std::isinf(scale)) scale = 1.0f / std::sqrt(static_cast<float>(d));
+
+  kvzip::ScoreArgs a;
+  a.q = q;
+  a.k_ctx = k_ctx;
+  a.k_self = k_self;
+  a.scores = scores;
+  a.status = static_cast<uint32_t*>(workspace);
+  a.lse2 = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kvzip::kScoreWsHeader);
+  a.B = B;
+  a.G = G;
+  a.n_in = n_in;
+  a.n_c = n_c;
+  a.d = d;
+  a.R = static_cast<int>(R);
+  a.R_pad = static_cast<int>(row_pad(R));
+  a.scale = scale;
+  a.timeout_ns = g_timeout_ns.load();
+  a.passes = passes;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int launches = 0;
+  cudaError_t e = (dt == KVZIP_BF16) ? kvzip::launch_score_tc(a, s, &launches)
+                                     : kvzip::launch_score_simt_f32(a, s, &launches);
+  if (e == cudaErrorInvalidValue) return KVZIP_ERR_INVALID_ARG;  // tensor map rejected the layout
+  if (e == cudaSuccess) g_last_launches.store(launches);
+  return from_cuda(e);
+}
+
+kvzip_status kvzip_score_chunk(kvzip_dtype dt, const void* q, const void* k_ctx,
+                               const void* k_self, float* scores, int B, int G, int n_in,
+                               int n_c, int d, float scale, void* workspace, size_t ws_bytes,
+                               void* stream) {
+  return score_passes(3, dt, q, k_ctx, k_self, scores, B, G, n_in, n_c, d, scale, workspace,
+                      ws_bytes, stream);
+}
+
+kvzip_status kvzip_score_lse(kvzip_dtype dt, const void* q, const void* k_ctx,
+                             const void* k_self, float* scores, int B, int G, int n_in, int n_c,
+                             int d, float scale, void* workspace, size_t ws_bytes, void* stream) {
+  return score_passes(1, dt, q, k_ctx, k_self, scores, B, G, n_in, n_c, d, scale, workspace,
+                      ws_bytes, stream);
+}
+
+kvzip_status kvzip_score_colmax(kvzip_dtype dt, const void* q, const void* k_ctx,
+                                const void* k_self, float* scores, int B, int G, int n_in,
+                                int n_c, int d, float scale, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  return score_passes(2, dt, q, k_ctx, k_self, scores, B, G, n_in, n_c, d, scale, workspace,
+                      ws_bytes, stream);
+}
+
+kvzip_status kvzip_workspace_status(void* workspace, void* stream) {
+  if (!workspace) return KVZIP_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return KVZIP_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return KVZIP_ERR_CUDA;
+  const uint32_t zero = 0;
+  if (cudaMemcpy(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+    return KVZIP_ERR_CUDA;
+  return (word & kvzip::kStatusTimeout) ? KVZIP_ERR_TIMEOUT : KVZIP_OK;
+}
+
+int64_t kvzip_keep_count(double r, int64_t N) {
+  if (!(r >= 0.0 && r <= 1.0) || N < 0) return -1;
+  return static_cast<int64_t>(std::ceil(r * static_cast<double>(N)));
+}
+
+size_t kvzip_select_workspace_size(int64_t N, int64_t n_heads) {
+  if (N < 0 || n_heads <= 0) return 0;
+  return kvzip::select_ws_bytes(N, n_heads);
+}
+
+kvzip_status kvzip_select(const float* scores, int64_t N, int64_t k, int64_t n_heads,
+                          uint8_t* keep, int64_t* offsets, float* threshold, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  if (N < 0 || n_heads <= 0 || k < 0 || k > N) return KVZIP_ERR_INVALID_ARG;
+  if (N % n_heads != 0 || N >= (int64_t{1} << 31) || n_heads > (int64_t{1} << 24))
+    return KVZIP_ERR_INVALID_ARG;
+  if (!offsets || !workspace || (N > 0 && (!scores || !keep))) return KVZIP_ERR_INVALID_ARG;
+  if (!aligned(offsets, 8) || (scores && !aligned(scores, 16)) || !aligned(workspace, 256) ||
+      (threshold && !aligned(threshold, 4)))
+    return KVZIP_ERR_INVALID_ARG;
+  if (ws_bytes < kvzip_select_workspace_size(N, n_heads)) return KVZIP_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (N == 0) {  // no scores: every head keeps nothing
+    cudaError_t e = cudaMemsetAsync(offsets, 0, sizeof(int64_t) * (n_heads + 1), s);
+    if (e == cudaSuccess && threshold) {
+      const float inf = INFINITY;
+      e = cudaMemcpyAsync(threshold, &inf, sizeof(float), cudaMemcpyHostToDevice, s);
+      if (e == cudaSuccess) e = cudaStreamSynchronize(s);  // `inf` lives on this stack frame
+    }
+    return from_cuda(e);
+  }
+  kvzip::SelectArgs a;
+  a.scores = scores;
+  a.N = N;
+  a.k = k;
+  a.n_heads = n_heads;
+  a.n_c = N / n_heads;
+  a.keep = keep;
+  a.offsets = offsets;
+  a.threshold = threshold;
+  a.ws = workspace;
+  a.ws_bytes = ws_bytes;
+  int launches = 0;
+  cudaError_t e = kvzip::launch_select(a, s, &launches);
+  if (e == cudaSuccess) g_last_launches.store(launches);
+  return from_cuda(e);
+}
+
+size_t kvzip_compact_workspace_size(int64_t n_heads, int n_c) {
+  if (n_heads <= 0 || n_c < 0) return 0;
+  return kvzip::compact_ws_bytes(n_heads, n_c);
+}
+
+kvzip_status kvzip_compact(const void* k, const void* v, const uint8_t* keep,
+                           const int64_t* offsets, int64_t n_heads, int n_c, int d, void* k_out,
+                           void* v_out, int32_t* pos_out, void* workspace, size_t ws_bytes,
+                           void* stream) {
+  if (n_heads <= 0 || n_c < 0 || n_heads > (int64_t{1} << 24)) return KVZIP_ERR_INVALID_ARG;
+  if (d != 128 && d != 256) return d > 0 ? KVZIP_ERR_UNSUPPORTED : KVZIP_ERR_INVALID_ARG;
+  if (n_c == 0) return KVZIP_OK;
+  if (n_heads * static_cast<int64_t>(n_c) >= (int64_t{1} << 31)) return KVZIP_ERR_UNSUPPORTED;
+  if (!k || !v || !keep || !offsets || !workspace) return KVZIP_ERR_INVALID_ARG;
+  if ((k_out == nullptr) != (v_out == nullptr)) return KVZIP_ERR_INVALID_ARG;
+  if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_out, 16) || !aligned(v_out, 16) ||
+      !aligned(offsets, 8) || !aligned(workspace, 256) || (pos_out && !aligned(pos_out, 4)))
+    return KVZIP_ERR_INVALID_ARG;
+  if (ws_bytes < kvzip_compact_workspace_size(n_heads, n_c)) return KVZIP_ERR_INVALID_ARG;
+  kvzip::CompactArgs a;
+  a.k = k;
+  a.v = v;
+  a.keep = keep;
+  a.offsets = offsets;
+  a.n_heads = n_heads;
+  a.n_c = n_c;
+  a.d = d;
+  a.k_out = k_out;
+  a.v_out = v_out;
+  a.pos_out = pos_out;
+  a.ws = workspace;
+  a.ws_bytes = ws_bytes;
+  int launches = 0;
+  cudaError_t e = kvzip::launch_compact(a, static_cast<cudaStream_t>(stream), &launches);
+  if (e == cudaSuccess) g_last_launches.store(launches);
+  return from_cuda(e);
+}
+
+}  // extern "C"

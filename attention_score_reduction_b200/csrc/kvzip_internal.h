@@ -1,0 +1,66 @@
+// Internal declarations shared by the host-side C ABI and the kernel files.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+namespace kvzip {
+
+// Status bits the kernels OR into the workspace header word.
+constexpr uint32_t kStatusTimeout = 1u;
+
+// Bytes reserved at the front of the scoring workspace for the status word.
+constexpr size_t kScoreWsHeader = 256;
+
+// Query rows of one unit are padded to this many in the log-sum-exp buffer.
+constexpr int kRowPad = 256;
+
+struct ScoreArgs {
+  const void* q;
+  const void* k_ctx;
+  const void* k_self;
+  float* scores;
+  float* lse2;        // [B][R_pad] base-2 log-sum-exp of the scaled logits
+  uint32_t* status;   // sticky status word
+  int B, G, n_in, n_c, d;
+  int R, R_pad;
+  float scale;
+  uint64_t timeout_ns;
+  int passes;         // bit 0: pass 1 (row log-sum-exp), bit 1: pass 2 (column max)
+};
+
+// Tensor-core (tcgen05) scorer for bf16 inputs.  Returns a cudaError_t.
+cudaError_t launch_score_tc(const ScoreArgs& a, cudaStream_t s, int* launches);
+// CUDA-core scorer for fp32 inputs.
+cudaError_t launch_score_simt_f32(const ScoreArgs& a, cudaStream_t s, int* launches);
+
+struct SelectArgs {
+  const float* scores;
+  int64_t N, k, n_heads, n_c;
+  uint8_t* keep;
+  int64_t* offsets;
+  float* threshold;
+  void* ws;
+  size_t ws_bytes;
+};
+size_t select_ws_bytes(int64_t N, int64_t n_heads);
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launches);
+
+struct CompactArgs {
+  const void* k;
+  const void* v;
+  const uint8_t* keep;
+  const int64_t* offsets;
+  int64_t n_heads;
+  int n_c, d;
+  void* k_out;
+  void* v_out;
+  int32_t* pos_out;
+  void* ws;
+  size_t ws_bytes;
+};
+size_t compact_ws_bytes(int64_t n_heads, int n_c);
+cudaError_t launch_compact(const CompactArgs& a, cudaStream_t s, int* launches);
+
+}  // namespace kvzip

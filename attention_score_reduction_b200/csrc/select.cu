@@ -1,0 +1,367 @@
+// Global top-k selection over all (layer, head, position) scores.
+//
+// KVzip evicts the lowest-scoring KV pairs once per context, ranking all
+// L x H x n_c scores together so that head budgets follow the scores (scime.ai
+// summary, "Approach" and the "Measured effects" row on non-uniform head
+// budgets; rebuttal: S has shape L x H x n_c).  The kept set is the k largest
+// scores; equal scores are taken lowest flat index first, so the mask is unique.
+//
+// Scores are finite and >= 0, so their IEEE bit patterns, read as uint32, sort
+// like the values.  The threshold tau (the k-th largest bit pattern) is found
+// by a three-round radix select on 11 + 11 + 10 bits; every round is one
+// histogram pass over HBM plus a one-block pick, all on the stream with no
+// host round trip.  A mask pass then writes keep[f] and per-block kept counts;
+// a one-block scan turns those into per-head offsets.  When more elements equal
+// tau than are still needed, a counting pass and a scan give every block the
+// number of equal elements before it, and ties are ranked in flat order.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+
+#include "kvzip_internal.h"
+
+namespace kvzip {
+
+namespace {
+
+constexpr int kSelThreads = 256;
+constexpr int kSelSeg = 8192;     // scores per block in the mask / tie passes
+constexpr int kHistThreads = 512;
+constexpr int kPickThreads = 1024;
+
+struct SelState {
+  uint32_t prefix;                // bits of tau fixed so far
+  uint32_t tau;                   // final threshold bit pattern
+  unsigned long long k_rem;       // rank still sought inside the current prefix class
+  unsigned long long count_gt;    // elements strictly above the current prefix class
+  unsigned long long n_eq;        // elements equal to tau
+  unsigned long long take_eq;     // of those, how many are kept
+  uint32_t keep_none;             // k == 0
+  uint32_t pad[5];
+};
+
+struct SelWs {
+  SelState* st;
+  uint32_t* hist;     // 2048 + 2048 + 1024 bins
+  uint32_t* blk_cnt;  // kept per mask block
+  uint32_t* blk_eq;   // equal-to-tau per mask block, scanned in place
+};
+
+// Radix rounds: bins, shift of the digit, bits fixed before the round, histogram offset.
+__host__ __device__ constexpr int hist_bins(int p) { return p == 2 ? 1024 : 2048; }
+__host__ __device__ constexpr int hist_shift(int p) { return p == 0 ? 21 : (p == 1 ? 10 : 0); }
+__host__ __device__ constexpr uint32_t hist_mask(int p) {
+  return p == 0 ? 0u : (p == 1 ? 0xFFE00000u : 0xFFFFFC00u);
+}
+__host__ __device__ constexpr int hist_off(int p) { return p * 2048; }
+constexpr int kHistTotal = 5120;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+int64_t segs_per_head(int64_t n_c) { return (n_c + kSelSeg - 1) / kSelSeg; }
+
+__global__ void sel_init(SelState* st, uint32_t* hist, unsigned long long k, float* threshold) {
+  for (int i = threadIdx.x; i < kHistTotal; i += blockDim.x) hist[i] = 0;
+  if (threadIdx.x == 0) {
+    if (k == 0 && threshold) *threshold = INFINITY;
+    st->prefix = 0;
+    st->tau = 0x7F800000u;  // +inf: nothing above it is finite
+    st->k_rem = k;
+    st->count_gt = 0;
+    st->n_eq = 0;
+    st->take_eq = 0;
+    st->keep_none = (k == 0);
+  }
+}
+
+template <int PASS>
+__global__ void __launch_bounds__(kHistThreads)
+    sel_hist(const float* __restrict__ s, int64_t N, const SelState* st, uint32_t* hist) {
+  constexpr int NB = hist_bins(PASS);
+  constexpr int SH = hist_shift(PASS);
+  constexpr uint32_t PM = hist_mask(PASS);
+  __shared__ uint32_t h[NB];
+  for (int i = threadIdx.x; i < NB; i += blockDim.x) h[i] = 0;
+  __syncthreads();
+  const uint32_t prefix = st->prefix;
+  const int64_t n4 = N / 4;
+  const uint4* s4 = reinterpret_cast<const uint4*>(s);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += stride) {
+    const uint4 u = __ldcs(s4 + i);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if ((w[e] & PM) == prefix) atomicAdd(&h[(w[e] >> SH) & (NB - 1)], 1u);
+  }
+  for (int64_t i = 4 * n4 + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < N;
+       i += stride) {
+    const uint32_t w = __float_as_uint(s[i]);
+    if ((w & PM) == prefix) atomicAdd(&h[(w >> SH) & (NB - 1)], 1u);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < NB; i += blockDim.x)
+    if (h[i]) atomicAdd(&hist[hist_off(PASS) + i], h[i]);
+}
+
+// Inclusive scan of one value per thread across a block of kPickThreads.
+__device__ unsigned long long block_incl_scan(unsigned long long v, unsigned long long* sm) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) sm[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    unsigned long long w = (lane < static_cast<int>(blockDim.x >> 5)) ? sm[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long n = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += n;
+    }
+    sm[lane] = w;
+  }
+  __syncthreads();
+  const unsigned long long add = warp ? sm[warp - 1] : 0;
+  __syncthreads();
+  return v + add;
+}
+
+// Find the bin (counting from the top) that holds the k_rem-th largest element.
+template <int PASS>
+__global__ void __launch_bounds__(kPickThreads)
+    sel_pick(SelState* st, const uint32_t* hist, float* threshold) {
+  constexpr int NB = hist_bins(PASS);
+  constexpr int PER = NB / kPickThreads;  // 2 or 1 bins per thread
+  __shared__ unsigned long long sm[32];
+  __shared__ int found_bin;
+  __shared__ unsigned long long found_above;
+  if (st->keep_none) return;
+  const uint32_t* h = hist + hist_off(PASS);
+  // thread t owns bins NB-1-PER*t ... NB-PER*(t+1) (descending)
+  unsigned long long mine = 0;
+  uint32_t cnt[PER];
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    cnt[j] = h[NB - 1 - (PER * threadIdx.x + j)];
+    mine += cnt[j];
+  }
+  const unsigned long long incl = block_incl_scan(mine, sm);
+  const unsigned long long excl = incl - mine;
+  const unsigned long long k_rem = st->k_rem;
+  if (threadIdx.x == 0) found_bin = -1;
+  __syncthreads();
+  if (excl < k_rem && k_rem <= incl) {
+    unsigned long long above = excl;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      if (above + cnt[j] >= k_rem) {
+        found_bin = NB - 1 - (PER * threadIdx.x + j);
+        found_above = above;
+        break;
+      }
+      above += cnt[j];
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && found_bin >= 0) {
+    const uint32_t bin = static_cast<uint32_t>(found_bin);
+    st->prefix |= bin << hist_shift(PASS);
+    st->count_gt += found_above;
+    st->k_rem = k_rem - found_above;
+    if (PASS == 2) {
+      st->tau = st->prefix;
+      st->n_eq = h[bin];
+      st->take_eq = st->k_rem;
+      if (threshold) *threshold = __uint_as_float(st->prefix);
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t warp_excl_prefix(bool flag, uint32_t* total) {
+  const uint32_t m = __ballot_sync(0xffffffffu, flag);
+  *total = __popc(m);
+  return __popc(m & ((1u << (threadIdx.x & 31)) - 1u));
+}
+
+// Count scores equal to tau per mask block (only when ties must be ranked).
+__global__ void __launch_bounds__(kSelThreads)
+    sel_eqcount(const float* __restrict__ s, int64_t n_c, int64_t segs, const SelState* st,
+                uint32_t* blk_eq) {
+  if (st->keep_none || st->take_eq == st->n_eq) return;
+  const int64_t blk = blockIdx.x;
+  const int64_t h = blk / segs, sg = blk % segs;
+  const int64_t j0 = sg * kSelSeg, j1 = imin64(j0 + kSelSeg, n_c);
+  const float* base = s + h * n_c;
+  const uint32_t tau = st->tau;
+  uint32_t c = 0;
+  for (int64_t j = j0 + threadIdx.x; j < j1; j += kSelThreads)
+    c += (__float_as_uint(base[j]) == tau);
+  __shared__ uint32_t red[kSelThreads / 32];
+  c = __reduce_add_sync(0xffffffffu, c);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t t = 0;
+    for (int w = 0; w < kSelThreads / 32; ++w) t += red[w];
+    blk_eq[blk] = t;
+  }
+}
+
+// Exclusive scan of per-block values, in place, one block.
+__global__ void __launch_bounds__(kPickThreads)
+    sel_scan_blocks(uint32_t* v, int64_t n, const SelState* st, int only_if_ties) {
+  if (only_if_ties && (st->keep_none || st->take_eq == st->n_eq)) return;
+  __shared__ unsigned long long sm[32];
+  __shared__ unsigned long long carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int64_t base = 0; base < n; base += kPickThreads) {
+    const int64_t i = base + threadIdx.x;
+    const unsigned long long x = (i < n) ? v[i] : 0;
+    const unsigned long long incl = block_incl_scan(x, sm);
+    const unsigned long long c0 = carry;
+    if (i < n) v[i] = static_cast<uint32_t>(c0 + incl - x);
+    __syncthreads();
+    if (threadIdx.x == kPickThreads - 1) carry = c0 + incl;
+    __syncthreads();
+  }
+}
+
+// keep[f] and kept count per block.
+__global__ void __launch_bounds__(kSelThreads)
+    sel_mask(const float* __restrict__ s, int64_t n_c, int64_t segs, const SelState* st,
+             const uint32_t* blk_eq_base, uint8_t* keep, uint32_t* blk_cnt) {
+  const int64_t blk = blockIdx.x;
+  const int64_t h = blk / segs, sg = blk % segs;
+  const int64_t j0 = sg * kSelSeg, j1 = imin64(j0 + kSelSeg, n_c);
+  const float* base = s + h * n_c;
+  uint8_t* kb = keep + h * n_c;
+  const bool none = st->keep_none != 0;
+  const uint32_t tau = st->tau;
+  const bool rank_ties = !none && st->take_eq != st->n_eq;
+  const unsigned long long take_eq = st->take_eq;
+  __shared__ uint32_t wsum[kSelThreads / 32];
+  __shared__ uint32_t red[kSelThreads / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  unsigned long long tie_before = rank_ties ? blk_eq_base[blk] : 0;
+  uint32_t kept = 0;
+  for (int64_t jb = j0; jb < j1; jb += kSelThreads) {
+    const int64_t j = jb + threadIdx.x;
+    const bool in = j < j1;
+    const uint32_t u = in ? __float_as_uint(base[j]) : 0u;
+    bool k = in && !none && u > tau;
+    const bool eq = in && !none && u == tau;
+    if (!rank_ties) {
+      k = k || eq;
+    } else {
+      // rank of this tie among all ties in flat order
+      uint32_t wt;
+      const uint32_t pre = warp_excl_prefix(eq, &wt);
+      if (lane == 0) wsum[warp] = wt;
+      __syncthreads();
+      uint32_t before = 0, total = 0;
+      for (int w = 0; w < kSelThreads / 32; ++w) {
+        before += (w < warp) ? wsum[w] : 0;
+        total += wsum[w];
+      }
+      k = k || (eq && tie_before + before + pre < take_eq);
+      tie_before += total;
+      __syncthreads();
+    }
+    if (in) kb[j] = k ? 1 : 0;
+    kept += k;
+  }
+  kept = __reduce_add_sync(0xffffffffu, kept);
+  if (lane == 0) red[warp] = kept;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t t = 0;
+    for (int w = 0; w < kSelThreads / 32; ++w) t += red[w];
+    blk_cnt[blk] = t;
+  }
+}
+
+// offsets[h] = kept in heads < h, from per-block counts (one block).
+__global__ void __launch_bounds__(kPickThreads)
+    sel_offsets(const uint32_t* blk_cnt, int64_t n_heads, int64_t segs, int64_t* offsets) {
+  __shared__ unsigned long long sm[32];
+  __shared__ unsigned long long carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int64_t base = 0; base < n_heads; base += kPickThreads) {
+    const int64_t h = base + threadIdx.x;
+    unsigned long long c = 0;
+    if (h < n_heads)
+      for (int64_t sg = 0; sg < segs; ++sg) c += blk_cnt[h * segs + sg];
+    const unsigned long long incl = block_incl_scan(c, sm);
+    const unsigned long long c0 = carry;
+    if (h < n_heads) offsets[h] = static_cast<int64_t>(c0 + incl - c);
+    __syncthreads();
+    if (threadIdx.x == kPickThreads - 1) carry = c0 + incl;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) offsets[n_heads] = static_cast<int64_t>(carry);
+}
+
+SelWs carve(void* ws, int64_t nblk) {
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  SelWs w;
+  w.st = reinterpret_cast<SelState*>(p);
+  p += 256;
+  w.hist = reinterpret_cast<uint32_t*>(p);
+  p += align_up(kHistTotal * 4, 256);
+  w.blk_cnt = reinterpret_cast<uint32_t*>(p);
+  p += align_up(static_cast<size_t>(nblk) * 4, 256);
+  w.blk_eq = reinterpret_cast<uint32_t*>(p);
+  return w;
+}
+
+}  // namespace
+
+size_t select_ws_bytes(int64_t N, int64_t n_heads) {
+  const int64_t n_c = n_heads > 0 ? N / n_heads : 0;
+  const int64_t nblk = n_heads * segs_per_head(n_c);
+  return 256 + align_up(kHistTotal * 4, 256) + 2 * align_up(static_cast<size_t>(nblk) * 4, 256);
+}
+
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launches) {
+  const int64_t segs = segs_per_head(a.n_c);
+  const int64_t nblk = a.n_heads * segs;
+  SelWs w = carve(a.ws, nblk);
+  int n = 0;
+  sel_init<<<1, 1024, 0, s>>>(w.st, w.hist, static_cast<unsigned long long>(a.k), a.threshold);
+  ++n;
+  if (a.k > 0) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t want = (a.N / 4 + kHistThreads - 1) / kHistThreads;
+    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, 4LL * sms)));
+    sel_hist<0><<<grid, kHistThreads, 0, s>>>(a.scores, a.N, w.st, w.hist);
+    sel_pick<0><<<1, kPickThreads, 0, s>>>(w.st, w.hist, a.threshold);
+    sel_hist<1><<<grid, kHistThreads, 0, s>>>(a.scores, a.N, w.st, w.hist);
+    sel_pick<1><<<1, kPickThreads, 0, s>>>(w.st, w.hist, a.threshold);
+    sel_hist<2><<<grid, kHistThreads, 0, s>>>(a.scores, a.N, w.st, w.hist);
+    sel_pick<2><<<1, kPickThreads, 0, s>>>(w.st, w.hist, a.threshold);
+    sel_eqcount<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs, w.st,
+                                                                   w.blk_eq);
+    sel_scan_blocks<<<1, kPickThreads, 0, s>>>(w.blk_eq, nblk, w.st, 1);
+    n += 8;
+  }
+  sel_mask<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs, w.st,
+                                                              w.blk_eq, a.keep, w.blk_cnt);
+  sel_offsets<<<1, kPickThreads, 0, s>>>(w.blk_cnt, a.n_heads, segs, a.offsets);
+  n += 2;
+  if (launches) *launches += n;
+  return cudaGetLastError();
+}
+
+}  // namespace kvzip

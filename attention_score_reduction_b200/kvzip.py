@@ -1,0 +1,226 @@
+"""ctypes binding of libkvzip (include/kvzip.h): argument marshalling only.
+
+Every computation runs in the library's CUDA kernels; torch tensors provide
+device memory and the stream.  If the library is missing, importing this
+module raises: there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkvzip.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
+BF16, F32 = 0, 1
+
+
+class KvzipError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libkvzip.so not found at {LIB_PATH}; build it with "
+            "`python -m attention_score_reduction_b200.build` (there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, sz, f32, f64, u64 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+                                       ctypes.c_size_t, ctypes.c_float, ctypes.c_double,
+                                       ctypes.c_uint64)
+    sig = {
+        "kvzip_score_workspace_size": (sz, [i32, i32, i32]),
+        "kvzip_score_chunk": (i32, [i32, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, sz, vp]),
+        "kvzip_score_lse": (i32, [i32, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, sz, vp]),
+        "kvzip_score_colmax": (i32, [i32, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, sz, vp]),
+        "kvzip_workspace_status": (i32, [vp, vp]),
+        "kvzip_set_wait_timeout_ns": (None, [u64]),
+        "kvzip_keep_count": (i64, [f64, i64]),
+        "kvzip_select_workspace_size": (sz, [i64, i64]),
+        "kvzip_select": (i32, [vp, i64, i64, i64, vp, vp, vp, vp, sz, vp]),
+        "kvzip_compact_workspace_size": (sz, [i64, i32]),
+        "kvzip_compact": (i32, [vp, vp, vp, vp, i64, i32, i32, vp, vp, vp, vp, sz, vp]),
+        "kvzip_last_launch_count": (i32, []),
+        "kvzip_status_string": (ctypes.c_char_p, [i32]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return _lib.kvzip_status_string(int(s)).decode()
+
+
+def _check(s: int, where: str):
+    if s != OK:
+        raise KvzipError(s, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _dev_contig(name, t, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+# ---------------------------------------------------------------- scoring
+
+def score_workspace_size(B: int, G: int, n_in: int) -> int:
+    return int(_lib.kvzip_score_workspace_size(B, G, n_in))
+
+
+def new_score_workspace(B: int, G: int, n_in: int, device=None) -> torch.Tensor:
+    """Zero-initialised workspace (the status word must start at 0)."""
+    n = score_workspace_size(B, G, n_in)
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def score_chunk(q: torch.Tensor, k_ctx: torch.Tensor, k_self: torch.Tensor, scores: torch.Tensor,
+                workspace: torch.Tensor | None = None, scale: float = 0.0, stream=None,
+                which: str = "both"):
+    """scores[b][j] = max(scores[b][j], max_rho softmax(...)[rho][j]) for one chunk.
+
+    q [B][G][n_in][d], k_ctx [B][n_c][d], k_self [B][n_in][d] (bf16 or fp32,
+    same dtype), scores [B][n_c] float32.  ``which`` = "both" (kvzip_score_chunk),
+    "lse" (kvzip_score_lse) or "colmax" (kvzip_score_colmax).
+    """
+    fn = {"both": _lib.kvzip_score_chunk, "lse": _lib.kvzip_score_lse,
+          "colmax": _lib.kvzip_score_colmax}[which]
+    for n, t in (("q", q), ("k_ctx", k_ctx), ("k_self", k_self)):
+        _dev_contig(n, t, q.dtype)
+    _dev_contig("scores", scores, torch.float32)
+    B, G, n_in, d = q.shape
+    n_c = k_ctx.shape[1]
+    if k_ctx.shape != (B, n_c, d) or k_self.shape != (B, n_in, d) or scores.shape != (B, n_c):
+        raise ValueError("shape mismatch between q, k_ctx, k_self and scores")
+    if workspace is None:
+        workspace = new_score_workspace(B, G, n_in, q.device)
+    s = fn(_dtype_code(q), _ptr(q), _ptr(k_ctx), _ptr(k_self), _ptr(scores), B, G, n_in, n_c, d,
+           float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(),
+           _stream(stream))
+    _check(s, "kvzip_score_" + which)
+    return scores
+
+
+def workspace_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise and return (and clear) the scoring status word (OK or ERR_TIMEOUT)."""
+    return int(_lib.kvzip_workspace_status(_ptr(workspace), _stream(stream)))
+
+
+def set_wait_timeout_ns(ns: int):
+    _lib.kvzip_set_wait_timeout_ns(int(ns))
+
+
+def read_lse(workspace: torch.Tensor, B: int, G: int, n_in: int) -> torch.Tensor:
+    """Natural-log row normalisers the last pass-1 launch left in the workspace,
+    [B][G*n_in] (a view into the workspace's padded buffer, converted)."""
+    R = G * n_in
+    R_pad = (R + 255) // 256 * 256
+    lse2 = workspace[256:256 + B * R_pad * 4].view(torch.float32).view(B, R_pad)[:, :R]
+    return lse2 * 0.6931471805599453
+
+
+# ---------------------------------------------------------------- selection
+
+def keep_count(r: float, N: int) -> int:
+    k = int(_lib.kvzip_keep_count(float(r), int(N)))
+    if k < 0:
+        raise ValueError("r must be in [0, 1] and N >= 0")
+    return k
+
+
+def select_workspace_size(N: int, n_heads: int) -> int:
+    return int(_lib.kvzip_select_workspace_size(N, n_heads))
+
+
+def select(scores: torch.Tensor, k: int, n_heads: int, keep: torch.Tensor | None = None,
+           offsets: torch.Tensor | None = None, threshold: torch.Tensor | None = None,
+           workspace: torch.Tensor | None = None, stream=None):
+    """Global top-k keep mask, per-head offsets and the threshold score.
+
+    Returns (keep uint8 [N], offsets int64 [n_heads+1], threshold float32 [1]).
+    """
+    _dev_contig("scores", scores, torch.float32)
+    N = scores.numel()
+    dev = scores.device
+    keep = torch.empty(N, dtype=torch.uint8, device=dev) if keep is None else keep
+    offsets = torch.empty(n_heads + 1, dtype=torch.int64, device=dev) if offsets is None else offsets
+    threshold = torch.empty(1, dtype=torch.float32, device=dev) if threshold is None else threshold
+    if workspace is None:
+        workspace = torch.empty(max(select_workspace_size(N, n_heads), 256), dtype=torch.uint8,
+                                device=dev)
+    s = _lib.kvzip_select(_ptr(scores), N, int(k), int(n_heads), _ptr(keep), _ptr(offsets),
+                          _ptr(threshold), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(s, "kvzip_select")
+    return keep, offsets, threshold
+
+
+# ---------------------------------------------------------------- compaction
+
+def compact_workspace_size(n_heads: int, n_c: int) -> int:
+    return int(_lib.kvzip_compact_workspace_size(n_heads, n_c))
+
+
+def compact(k: torch.Tensor, v: torch.Tensor, keep: torch.Tensor, offsets: torch.Tensor,
+            total: int, k_out: torch.Tensor | None = None, v_out: torch.Tensor | None = None,
+            pos_out: torch.Tensor | None = None, want_pos: bool = True,
+            workspace: torch.Tensor | None = None, stream=None):
+    """Pack kept rows per head.  ``total`` = offsets[-1] (known on the host as k).
+
+    Returns (k_out [total][d], v_out [total][d], pos_out int32 [total] or None).
+    """
+    _dev_contig("k", k, torch.bfloat16)
+    _dev_contig("v", v, torch.bfloat16)
+    n_heads, n_c, d = k.shape
+    dev = k.device
+    k_out = torch.empty(total, d, dtype=k.dtype, device=dev) if k_out is None else k_out
+    v_out = torch.empty(total, d, dtype=v.dtype, device=dev) if v_out is None else v_out
+    if pos_out is None and want_pos:
+        pos_out = torch.empty(total, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(compact_workspace_size(n_heads, n_c), 256), dtype=torch.uint8,
+                                device=dev)
+    s = _lib.kvzip_compact(_ptr(k), _ptr(v), _ptr(keep), _ptr(offsets), n_heads, n_c, d,
+                           _ptr(k_out), _ptr(v_out), _ptr(pos_out), _ptr(workspace),
+                           workspace.numel(), _stream(stream))
+    _check(s, "kvzip_compact")
+    return k_out, v_out, pos_out
+
+
+def last_launch_count() -> int:
+    return int(_lib.kvzip_last_launch_count())

@@ -1,0 +1,141 @@
+"""End-to-end KVzip compression of one context: chunked scoring, global top-r
+selection and per-head compaction, through libkvzip.
+
+This is the user-facing call.  ``Compressor`` owns the device buffers for one
+context shape and runs the three C-ABI calls on a CUDA stream:
+
+  1. ``kvzip_score_chunk`` once per reconstruction chunk (blog post section
+     4.5: chunked scoring keeps memory linear in n_c), merging into the
+     L x H x n_c score tensor by a running max;
+  2. ``kvzip_select`` once per context (scime.ai summary, "Approach": evict the
+     lowest-scoring pairs once, query-agnostically), global over (l, h, j);
+  3. ``kvzip_compact`` once, packing the kept K/V rows per head.
+
+``compress_from_host`` is the same path for inputs that start in (pinned)
+host memory: the context K/V and each chunk's Q / K_self are uploaded on a
+copy stream that runs ahead of the scorer, and the compacted cache is read
+back.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import kvzip as kz
+
+
+@dataclass
+class Compressed:
+    k: torch.Tensor          # [kept][d]   packed head-major, positions ascending per head
+    v: torch.Tensor          # [kept][d]
+    pos: torch.Tensor        # [kept] int32 positions within the head
+    offsets: torch.Tensor    # [units + 1] int64; head h owns rows offsets[h]:offsets[h+1]
+    kept: int                # = offsets[-1]
+    threshold: torch.Tensor  # [1] float32, the kept-th largest score
+
+
+class Compressor:
+    """Device state for compressing contexts of one shape.
+
+    units = L * H (layer-major), n_c context keys per unit, head dim d, G
+    query heads per KV head, max_n_in = largest chunk (prompt + context rows).
+    """
+
+    def __init__(self, units: int, n_c: int, d: int, G: int, max_n_in: int, device="cuda"):
+        self.units, self.n_c, self.d, self.G, self.max_n_in = units, n_c, d, G, max_n_in
+        self.device = torch.device(device)
+        N = units * n_c
+        self.scores = torch.zeros(units, n_c, dtype=torch.float32, device=self.device)
+        self.score_ws = kz.new_score_workspace(units, G, max_n_in, self.device)
+        self.select_ws = torch.empty(max(kz.select_workspace_size(N, units), 256),
+                                     dtype=torch.uint8, device=self.device)
+        self.compact_ws = torch.empty(max(kz.compact_workspace_size(units, n_c), 256),
+                                      dtype=torch.uint8, device=self.device)
+        self.keep = torch.empty(N, dtype=torch.uint8, device=self.device)
+        self.offsets = torch.empty(units + 1, dtype=torch.int64, device=self.device)
+        self.threshold = torch.empty(1, dtype=torch.float32, device=self.device)
+        self.launches = 0
+
+    def reset(self):
+        self.scores.zero_()
+
+    def score_chunk(self, q, k_ctx, k_self, scale: float = 0.0, stream=None):
+        kz.score_chunk(q, k_ctx, k_self, self.scores, self.score_ws, scale, stream)
+        self.launches += kz.last_launch_count()
+
+    def select(self, r: float, stream=None) -> int:
+        kept = kz.keep_count(r, self.scores.numel())
+        kz.select(self.scores.view(-1), kept, self.units, self.keep, self.offsets, self.threshold,
+                  self.select_ws, stream)
+        self.launches += kz.last_launch_count()
+        return kept
+
+    def compact(self, k_ctx, v, kept: int, k_out=None, v_out=None, pos_out=None, stream=None):
+        out = kz.compact(k_ctx, v, self.keep, self.offsets, kept, k_out, v_out, pos_out,
+                         workspace=self.compact_ws, stream=stream)
+        self.launches += kz.last_launch_count()
+        return out
+
+    def compress(self, k_ctx, v, chunks, r: float, scale: float = 0.0, stream=None,
+                 out=None) -> Compressed:
+        """k_ctx, v: [units][n_c][d] bf16 on the device; chunks: iterable of
+        (q [units][G][n_in][d], k_self [units][n_in][d]) device tensors."""
+        self.reset()
+        for q, ks in chunks:
+            self.score_chunk(q, k_ctx, ks, scale, stream)
+        kept = self.select(r, stream)
+        k_out, v_out, pos = self.compact(k_ctx, v, kept, *(out or (None, None, None)),
+                                         stream=stream)
+        return Compressed(k_out, v_out, pos, self.offsets, kept, self.threshold)
+
+    def check_status(self, stream=None):
+        s = kz.workspace_status(self.score_ws, stream)
+        if s != kz.OK:
+            raise kz.KvzipError(s, "scoring kernels")
+
+
+def compress_from_host(comp: Compressor, k_ctx_h, v_h, q_chunks_h, ks_chunks_h, r: float,
+                       dev_bufs: dict, host_out: dict | None = None, scale: float = 0.0):
+    """Upload host inputs, compress, and read the compacted cache back.
+
+    k_ctx_h, v_h: pinned host [units][n_c][d]; q_chunks_h / ks_chunks_h: lists of
+    pinned host chunk tensors.  ``dev_bufs`` holds reusable device tensors
+    ("k_ctx", "v", and lists "q", "ks" of per-chunk buffers).  ``host_out``
+    (pinned) receives "k", "v", "pos", "offsets".  Uploads run on a side
+    stream, each chunk's upload recorded by an event the scorer waits on.
+    Returns (Compressed on the device, host_out, bytes_h2d, bytes_d2h).
+    """
+    main = torch.cuda.current_stream()
+    copy = dev_bufs.setdefault("_copy_stream", torch.cuda.Stream())
+    copy.wait_stream(main)          # device buffers are free once earlier work is done
+    h2d = 0
+    with torch.cuda.stream(copy):
+        dev_bufs["k_ctx"].copy_(k_ctx_h, non_blocking=True)
+        dev_bufs["v"].copy_(v_h, non_blocking=True)
+        h2d += k_ctx_h.numel() * k_ctx_h.element_size() + v_h.numel() * v_h.element_size()
+        ev_kv = torch.cuda.Event()
+        ev_kv.record(copy)
+        evs = []
+        for qd, ksd, qh, ksh in zip(dev_bufs["q"], dev_bufs["ks"], q_chunks_h, ks_chunks_h):
+            qd.copy_(qh, non_blocking=True)
+            ksd.copy_(ksh, non_blocking=True)
+            h2d += qh.numel() * qh.element_size() + ksh.numel() * ksh.element_size()
+            e = torch.cuda.Event()
+            e.record(copy)
+            evs.append(e)
+    comp.reset()
+    main.wait_event(ev_kv)
+    for qd, ksd, e in zip(dev_bufs["q"], dev_bufs["ks"], evs):
+        main.wait_event(e)
+        comp.score_chunk(qd, dev_bufs["k_ctx"], ksd, scale)
+    kept = comp.select(r)
+    k_out, v_out, pos = comp.compact(dev_bufs["k_ctx"], dev_bufs["v"], kept)
+    d2h = 0
+    if host_out is not None:
+        host_out["k"][:kept].copy_(k_out, non_blocking=True)
+        host_out["v"][:kept].copy_(v_out, non_blocking=True)
+        host_out["pos"][:kept].copy_(pos, non_blocking=True)
+        host_out["offsets"].copy_(comp.offsets, non_blocking=True)
+        d2h = (k_out.numel() * 2 + v_out.numel() * 2 + pos.numel() * 4 + comp.offsets.numel() * 8)
+    return Compressed(k_out, v_out, pos, comp.offsets, kept, comp.threshold), host_out, h2d, d2h

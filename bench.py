@@ -1,0 +1,378 @@
+#!/usr/bin/env python
+"""KVzip scoring -> global top-r selection -> per-head compaction on B200.
+
+One step = one whole context through the hot path: every reconstruction chunk
+scored for all L x H units (two tensor-core passes per chunk), one global
+selection over the L x H x n_c scores, one compaction of the kept K/V rows.
+Default workload: LLaMA3.1-8B KV shape (32 layers x 8 KV heads, G = 4, d = 128)
+with a 131072-token context scored in 64 chunks of 2048 (+16 prompt rows), r = 0.3.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Inputs are synthetic (seeded) and resident in
+HBM for ``value``; ``e2e`` repeats the step from pinned host buffers through
+``pipeline.compress_from_host`` with the uploads and the read-back inside the
+timed region.  Under torchrun every rank compresses its own context (weak
+scaling); times are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from attention_score_reduction_b200 import benchutil as bu  # noqa: E402
+from attention_score_reduction_b200 import synth  # noqa: E402
+
+METRIC = "context tokens scored/sec (all layers+heads) @LLaMA3.1-8B 128K; % bf16 TC peak"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama8b_128k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--r", type=float, default=None, help="kept fraction (default: first of workload)")
+    ap.add_argument("--chunk", type=int, default=None, help="override context rows per chunk")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    return ap.parse_args()
+
+
+def workload(args, rank=0):
+    wl = synth.WORKLOADS[args.workload]
+    if args.chunk:
+        wl = wl.with_(m=args.chunk)
+    if rank:
+        wl = wl.with_(cfg_id=wl.cfg_id + bu.rank_salt(rank))
+    return wl
+
+
+def config_dict(wl, r):
+    return {"workload": wl.name, "L": wl.L, "H": wl.H, "G": wl.G, "d": wl.d, "n_c": wl.n_c,
+            "chunk": wl.m, "prompt_rows": wl.P, "chunks": wl.n_chunks, "r": r,
+            "inputs": "synthetic, seeded; " + _recipe(wl),
+            "l2": "inputs larger than L2 (K_ctx alone is %.1f GB per step)"
+                  % (wl.units * wl.n_c * wl.d * 2 / 1e9)}
+
+
+def _recipe(wl):
+    parts = ["Q,K,V ~ N(0,1) bf16" if wl.dtype == "bf16" else "Q,K ~ N(0,1) fp32"]
+    if wl.hi_frac:
+        parts.append(f"{wl.hi_frac:.0%} of key rows x{wl.hi_scale:g}")
+    if wl.sinks:
+        parts.append(f"first {wl.sinks} keys x{wl.sink_scale:g}")
+    if wl.lognormal_sigma:
+        parts.append(f"key rows x lognormal(0,{wl.lognormal_sigma:g})")
+    return ", ".join(parts)
+
+
+# ----------------------------------------------------------------- oracle sample
+
+def oracle_sample(wl, k_ctx_u, k_bits, q_g, ks_u, scores_layer, r):
+    """Time the CPU oracle on a bounded sample and extrapolate to one step.
+
+    Scoring sample: one (layer, head) unit, one chunk, one query head (n_in rows
+    against all n_c context keys + causal self keys); a step has units x chunks
+    x G such pieces.  Selection + compaction sample: one layer (H units); a step
+    has L of them.  Returns (seconds per step extrapolated, sample text, threads).
+    """
+    import numpy as np
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    s_c, _ = oracle.unit_chunk_scores(q_g, k_ctx_u, ks_u)
+    t_score = time.perf_counter() - t0
+    assert np.all(s_c > 0)
+    t0 = time.perf_counter()
+    kk = oracle.keep_count(r, scores_layer.size)
+    keep, off, _ = oracle.select(scores_layer.reshape(-1), kk, wl.H)
+    kv = np.broadcast_to(k_bits[None], (wl.H,) + k_bits.shape)   # H heads of bf16 rows
+    oracle.compact(kv, kv, keep, off)
+    t_sel = time.perf_counter() - t0
+    pieces = wl.units * wl.n_chunks * wl.G
+    step_s = t_score * pieces + t_sel * wl.L
+    sample = (f"scoring: 1 unit x 1 chunk x 1 of {wl.G} query heads ({q_g.shape[1]} rows x "
+              f"{wl.n_c}+self keys) in {t_score:.2f} s, x{pieces} extrapolated; "
+              f"select+compact: 1 layer ({wl.H} heads) in {t_sel:.2f} s, x{wl.L} extrapolated")
+    return step_s, sample, threads
+
+
+def sample_inputs(wl, r):
+    """Host float64 / int16 inputs of the oracle sample (chunk 0, unit 0, query head 0)."""
+    import numpy as np
+    k_ctx = synth.context_keys(wl, units=1)[0]
+    q, ks = synth.chunk_qk(wl, 0, units=1)
+    q_g = q[0, :1].double().numpy()
+    ks_u = ks[0].double().numpy()
+    k_u = k_ctx.double().numpy()
+    k_bits = k_ctx.view(torch.int16).numpy() if k_ctx.dtype == torch.bfloat16 else k_ctx.numpy()
+    rng = np.random.default_rng(0)
+    scores_layer = (rng.random((wl.H, wl.n_c)) ** 4).astype(np.float32)
+    return k_u, k_bits, q_g, ks_u, scores_layer
+
+
+def run_reference(args):
+    rank, world, _ = bu.dist_env()
+    if rank != 0:
+        return
+    wl = workload(args)
+    r = args.r if args.r is not None else wl.r[0]
+    import numpy as np
+    k_u, k_bits, q_g, ks_u, sl = sample_inputs(wl, r)
+    times, sample, threads = [], "", 1
+    for i in range(args.warmup + args.steps):
+        step_s, sample, threads = oracle_sample(wl, k_u, k_bits, q_g, ks_u, sl, r)
+        if i >= args.warmup:
+            times.append(step_s)
+    step_s = float(np.mean(times))
+    value = wl.n_c / step_s
+    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "config": config_dict(wl, r), "impl": "reference",
+           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+# ----------------------------------------------------------------- our arm
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    rank, world, local = bu.dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    from attention_score_reduction_b200 import kvzip as kz
+    from attention_score_reduction_b200 import pipeline
+
+    wl = workload(args, rank)
+    r = args.r if args.r is not None else wl.r[0]
+    dev = torch.device("cuda", local)
+    k_ctx, v = synth.context_kv(wl, device=dev)
+    chunks = [synth.chunk_qk(wl, c, device=dev) for c in range(wl.n_chunks)]
+    max_n_in = max(q.shape[2] for q, _ in chunks)
+    comp = pipeline.Compressor(wl.units, wl.n_c, wl.d, wl.G, max_n_in, device=dev)
+    N = wl.units * wl.n_c
+    kept = kz.keep_count(r, N)
+    k_out = torch.empty(kept, wl.d, dtype=torch.bfloat16, device=dev)
+    v_out = torch.empty_like(k_out)
+    pos_out = torch.empty(kept, dtype=torch.int32, device=dev)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+    per_chunk = []  # (ev0, ev1, ev2) per chunk, per timed step
+    stage_ev = []
+
+    def step(timed: bool):
+        comp.reset()
+        launches = 0
+        for q, ks in chunks:
+            if timed:
+                e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+                e0.record(stream)
+            kz.score_chunk(q, k_ctx, ks, comp.scores, comp.score_ws, which="lse")
+            launches += kz.last_launch_count()
+            if timed:
+                e1.record(stream)
+            kz.score_chunk(q, k_ctx, ks, comp.scores, comp.score_ws, which="colmax")
+            launches += kz.last_launch_count()
+            if timed:
+                e2.record(stream)
+                per_chunk.append((e0, e1, e2, q.shape[2]))
+        if timed:
+            s0, s1, s2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            s0.record(stream)
+        comp.select(r)
+        launches += kz.last_launch_count()
+        if timed:
+            s1.record(stream)
+        comp.compact(k_ctx, v, kept, k_out, v_out, pos_out)
+        launches += kz.last_launch_count()
+        if timed:
+            s2.record(stream)
+            stage_ev.append((s0, s1, s2))
+        return launches
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    comp.check_status()
+
+    bu.barrier(world)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    launches = 0
+    with bu.ClockSampler(local) as clk:
+        start.record(stream)
+        for _ in range(args.steps):
+            launches += step(True)
+        end.record(stream)
+        torch.cuda.synchronize()
+    bu.barrier(world)
+    comp.check_status()
+    clocks = clk.summary()
+    elapsed_ms = bu.max_over_ranks(start.elapsed_time(end), world, dev)
+    ms_per_step = elapsed_ms / args.steps
+    value = world * wl.n_c / (ms_per_step / 1e3)
+
+    # per-kernel device times
+    p1 = [a.elapsed_time(b) for a, b, _, _ in per_chunk]
+    p2 = [b.elapsed_time(c) for _, b, c, _ in per_chunk]
+    sel = [a.elapsed_time(b) for a, b, _ in stage_ev]
+    cmp = [b.elapsed_time(c) for _, b, c in stage_ev]
+    peaks = bu.load_peaks(os.path.join(ROOT, "MEASURED_PEAKS.json"))
+    fl = [bu.score_flops(wl.units, wl.G, n_in, wl.n_c, wl.d) for *_, n_in in per_chunk]
+    f1 = sum(f["pass1"] for f in fl) / len(fl)
+    f2 = sum(f["pass2"] for f in fl) / len(fl)
+    t1, t2 = sum(p1) / len(p1), sum(p2) / len(p2)
+    tf1, tf2 = f1 / (t1 * 1e-3) / 1e12, f2 / (t2 * 1e-3) / 1e12
+    peak_tf = peaks["bf16_tflops_sustained"]
+    dominant = "score_pass1_lse" if sum(p1) >= sum(p2) else "score_pass2_colmax"
+    dom_tf, dom_f = (tf1, f1) if dominant == "score_pass1_lse" else (tf2, f2)
+    # selection / compaction bytes: scores read once + mask written; kept K and V rows
+    # read and written once, positions written, mask read once.
+    sel_bytes = N * 4 + N
+    cmp_bytes = N + kept * wl.d * 2 * 2 * 2 + kept * 4
+    t_sel, t_cmp = sum(sel) / len(sel), sum(cmp) / len(cmp)
+    score_ms = (sum(p1) + sum(p2)) / args.steps
+    executed_tf = (f1 + f2) * len(p1) / args.steps / (ms_per_step * 1e-3) / 1e12
+    roofline = {"kernel": dominant, "bound": "tensor", "achieved": dom_tf, "peak": peak_tf,
+                "unit": "TFLOP/s", "frac": dom_tf / peak_tf, "traffic": None,
+                "peak_source": f"{peaks['source']} bf16 sustained",
+                "flops_per_launch": dom_f}
+    kernels = {
+        "score_pass1_lse": {"ms": t1, "tflops": tf1, "frac_of_peak": tf1 / peak_tf},
+        "score_pass2_colmax": {"ms": t2, "tflops": tf2, "frac_of_peak": tf2 / peak_tf},
+        "select": {"ms": t_sel, "gbs": sel_bytes / (t_sel * 1e-3) / 1e9,
+                   "frac_of_hbm": sel_bytes / (t_sel * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "compact": {"ms": t_cmp, "gbs": cmp_bytes / (t_cmp * 1e-3) / 1e9,
+                    "frac_of_hbm": cmp_bytes / (t_cmp * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "select_plus_compact_frac_of_hbm":
+            (sel_bytes + cmp_bytes) / ((t_sel + t_cmp) * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "scoring_ms_per_step": score_ms,
+        "scoring_pct_bf16_tc_peak": 100.0 * (f1 + f2) * len(p1) / args.steps
+                                     / (score_ms * 1e-3) / 1e12 / peak_tf,
+        "step_pct_bf16_tc_peak": 100.0 * executed_tf / peak_tf,
+    }
+
+    # ------------------------------------------------------------ end to end
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, wl, r, comp, k_ctx, v, chunks, kept, world, dev)
+
+    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+           "data": "synthetic", "config": config_dict(wl, r), "parallelism":
+           f"{world} independent contexts, one per GPU", "clocks": clocks,
+           "gpu_launches": launches, "roofline": roofline, "kernels": kernels,
+           "pct_bf16_tc_peak": kernels["step_pct_bf16_tc_peak"], "e2e": e2e}
+
+    # free device memory before the CPU baseline allocates host buffers
+    del chunks, k_ctx, v, comp
+    torch.cuda.empty_cache()
+    if world == 1 and rank == 0 and not args.no_cpu:
+        k_u, k_bits, q_g, ks_u, sl = sample_inputs(workload(args), r)
+        step_s, sample, threads = oracle_sample(wl, k_u, k_bits, q_g, ks_u, sl, r)
+        out["cpu_baseline"] = {"value": wl.n_c / step_s, "unit": "tokens/s", "cores": threads,
+                               "kind": "oracle", "sample": sample}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def _pinned_like(t):
+    """Page-locked host copy of a device tensor (registered in place, no size rounding)."""
+    h = torch.empty(t.shape, dtype=t.dtype)
+    h.copy_(t)
+    err = torch.cuda.cudart().cudaHostRegister(h.data_ptr(), h.numel() * h.element_size(), 0)
+    if int(err) != 0:
+        raise RuntimeError(f"cudaHostRegister failed ({int(err)})")
+    return h
+
+
+def _unpin(ts):
+    for h in ts:
+        torch.cuda.cudart().cudaHostUnregister(h.data_ptr())
+
+
+def run_e2e(args, wl, r, comp, k_ctx, v, chunks, kept, world, dev):
+    """Same step from pinned host memory: uploads, scoring, selection, compaction
+    and the read-back of the compacted cache all inside the timed region.
+
+    The host holds K_ctx, V and as many distinct chunk inputs as a host-memory
+    budget allows (all of them on a single-GPU run with enough RAM); when it
+    holds fewer, chunks reuse host buffers cyclically, so every chunk is still
+    uploaded in full each step."""
+    import psutil
+    from attention_score_reduction_b200 import pipeline
+    steps = args.e2e_steps or max(1, args.steps)
+    per_chunk = sum(t.numel() * t.element_size() for t in chunks[0])
+    fixed = 2 * k_ctx.numel() * k_ctx.element_size() + 2 * kept * wl.d * 2
+    budget = 0.6 * psutil.virtual_memory().available / world
+    n_host = int(max(1, min(len(chunks), (budget - fixed) // max(per_chunk, 1))))
+    k_h, v_h = _pinned_like(k_ctx), _pinned_like(v)
+    q_h = [_pinned_like(chunks[c][0]) for c in range(n_host)]
+    ks_h = [_pinned_like(chunks[c][1]) for c in range(n_host)]
+    qs = [q_h[c % n_host] for c in range(len(chunks))]
+    kss = [ks_h[c % n_host] for c in range(len(chunks))]
+    bufs = {"k_ctx": k_ctx, "v": v, "q": [q for q, _ in chunks], "ks": [ks for _, ks in chunks]}
+    host_out = {"k": torch.empty(kept, wl.d, dtype=torch.bfloat16),
+                "v": torch.empty(kept, wl.d, dtype=torch.bfloat16),
+                "pos": torch.empty(kept, dtype=torch.int32),
+                "offsets": torch.empty(wl.units + 1, dtype=torch.int64)}
+    for t in host_out.values():
+        torch.cuda.cudart().cudaHostRegister(t.data_ptr(), t.numel() * t.element_size(), 0)
+    stream = torch.cuda.current_stream()
+    h2d = d2h = 0
+    pipeline.compress_from_host(comp, k_h, v_h, qs, kss, r, bufs, host_out)  # warm-up
+    torch.cuda.synchronize()
+    bu.barrier(world)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        _, _, h2d, d2h = pipeline.compress_from_host(comp, k_h, v_h, qs, kss, r, bufs, host_out)
+    end.record(stream)
+    torch.cuda.synchronize()
+    bu.barrier(world)
+    comp.check_status()
+    assert int(host_out["offsets"][-1]) == kept
+    ms = bu.max_over_ranks(start.elapsed_time(end), world, dev) / steps
+    _unpin([k_h, v_h] + q_h + ks_h + list(host_out.values()))
+    return {"value": world * wl.n_c / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+            "steps": steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "host_chunk_buffers": n_host}
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,183 @@
+/*
+ * kvzip.h -- C ABI of libkvzip: KVzip query-agnostic KV importance scoring,
+ * global top-r selection and per-head KV compaction on one NVIDIA B200 (sm_100a).
+ *
+ * The method (KVzip: Query-Agnostic KV Cache Compression with Context
+ * Reconstruction, Kim et al.; blog post sections 4.1-4.5, the scime.ai summary's
+ * "Approach" paragraph and the authors' OpenReview rebuttal):
+ *
+ *   1. Per layer l and KV head h, the reconstruction queries Q_{l,h} in
+ *      R^{G x n_in x d} of one chunk attend to the prefilled context keys
+ *      K_c in R^{n_c x d} plus the chunk's own causal keys (blog post 4.3.1;
+ *      rebuttal: "2x attention FLOPs relative to prefilling").
+ *   2. Each context key j is scored by the largest softmax probability any
+ *      query row gives it, S_{l,h}[j] = max_{g,i} softmax(Q K^T / sqrt(d))[g,i,j]
+ *      (blog post 4.3.2), merged over chunks by a running max (4.5).
+ *   3. The top fraction r of all L x H x n_c scores is kept (rebuttal: S has
+ *      shape L x H x n_c), which leaves non-uniform per-head budgets (scime.ai
+ *      "Measured effects" table), and the kept K/V rows are packed per head
+ *      (blog post 4.1, step 5).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers (cudaMalloc / torch CUDA memory)
+ *     owned by the caller.  The library never allocates, frees or copies
+ *     caller memory, and never synchronises except in kvzip_workspace_status.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously on it.
+ *   - Arguments are validated on the host before anything is enqueued; a
+ *     rejected call enqueues nothing and returns KVZIP_ERR_INVALID_ARG (or
+ *     KVZIP_ERR_UNSUPPORTED for a valid but unimplemented shape).
+ *   - A failed launch returns KVZIP_ERR_CUDA.
+ *   - Device pointers must be 16-byte aligned unless stated otherwise.
+ *   - Calls that share a workspace must not overlap on the GPU.
+ */
+#ifndef KVZIP_H_
+#define KVZIP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KVZIP_OK = 0,
+  KVZIP_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, short workspace */
+  KVZIP_ERR_UNSUPPORTED = 2,   /* well-formed but not implemented (e.g. head dim 64) */
+  KVZIP_ERR_CUDA = 3,          /* a CUDA runtime/driver call or launch failed */
+  KVZIP_ERR_TIMEOUT = 4        /* a kernel gave up waiting on its own pipeline */
+} kvzip_status;
+
+typedef enum {
+  KVZIP_BF16 = 0,              /* bfloat16 Q / K (tensor-core path) */
+  KVZIP_F32 = 1                /* float32 Q / K (CUDA-core path) */
+} kvzip_dtype;
+
+/* ------------------------------------------------------------------ scoring */
+
+/* Bytes of workspace kvzip_score_chunk needs for B units of G*n_in query rows:
+ * a 256-byte status header plus one float per query row, rows padded to 256. */
+size_t kvzip_score_workspace_size(int B, int G, int n_in);
+
+/*
+ * Score one reconstruction chunk for B (layer, head) units and merge it into
+ * `scores` by a running maximum (blog post 4.3.1, 4.3.2, 4.5).
+ *
+ *   q       [B][G][n_in][d]  dtype `dt`; query row rho = g*n_in + i, i.e. the
+ *                            i-th token of the chunk (repeat-prompt tokens first,
+ *                            then the chunk's context tokens) for query head g.
+ *   k_ctx   [B][n_c][d]      dtype `dt`; the prefilled context keys K_c.
+ *   k_self  [B][n_in][d]     dtype `dt`; the chunk's own keys; row i sees self
+ *                            keys 0..i (causal, diagonal included).
+ *   scores  [B][n_c] float32, read-modify-write:
+ *             scores[b][j] = max(scores[b][j], max_rho P[b][rho][j]) where
+ *             P[b][rho][:] = softmax over (n_c context logits, i+1 self logits)
+ *             of scale * q . k.  Zero it before the first chunk; 4-byte aligned.
+ *   scale   <= 0 or NaN selects 1/sqrt(d).
+ *   d       128 or 256.
+ *   workspace / ws_bytes: >= kvzip_score_workspace_size(B, G, n_in) bytes,
+ *           256-byte aligned; its first 256 bytes are a sticky status word
+ *           that must be zeroed before first use (cudaMemsetAsync) and is read
+ *           and cleared by kvzip_workspace_status.
+ *
+ * B, G, n_in or n_c equal to 0 is a no-op.  Chunks may be scored in any order
+ * and re-scoring a chunk leaves `scores` unchanged (max is idempotent), so a
+ * caller can checkpoint `scores` between chunks.
+ */
+kvzip_status kvzip_score_chunk(kvzip_dtype dt, const void* q, const void* k_ctx,
+                               const void* k_self, float* scores, int B, int G,
+                               int n_in, int n_c, int d, float scale, void* workspace,
+                               size_t ws_bytes, void* stream);
+
+/* The two halves of kvzip_score_chunk, same arguments, for callers that time
+ * or schedule them separately.  kvzip_score_lse writes each query row's
+ * log-sum-exp over its context and visible self keys into the workspace
+ * (`scores` is not touched); kvzip_score_colmax then reads them and merges the
+ * chunk's per-key maxima into `scores`.  kvzip_score_chunk == lse, then
+ * colmax, on the same workspace and stream. */
+kvzip_status kvzip_score_lse(kvzip_dtype dt, const void* q, const void* k_ctx,
+                             const void* k_self, float* scores, int B, int G, int n_in,
+                             int n_c, int d, float scale, void* workspace, size_t ws_bytes,
+                             void* stream);
+kvzip_status kvzip_score_colmax(kvzip_dtype dt, const void* q, const void* k_ctx,
+                                const void* k_self, float* scores, int B, int G, int n_in,
+                                int n_c, int d, float scale, void* workspace, size_t ws_bytes,
+                                void* stream);
+
+/* Synchronise `stream`, then report (and clear) the status word the scoring
+ * kernels leave in `workspace`: KVZIP_OK, or KVZIP_ERR_TIMEOUT when a kernel
+ * abandoned a pipeline wait (its scores for that call are then incomplete). */
+kvzip_status kvzip_workspace_status(void* workspace, void* stream);
+
+/* Longest a scoring kernel waits on one pipeline stage before it gives up,
+ * records KVZIP_ERR_TIMEOUT in its workspace and returns (default 2 s).
+ * Applies to launches enqueued after the call; process-wide.  0 restores the
+ * default.  Intended for tests of the timeout path. */
+void kvzip_set_wait_timeout_ns(uint64_t ns);
+
+/* ---------------------------------------------------------------- selection */
+
+/* k = ceil(r * N), the product taken in IEEE double; -1 if r is outside
+ * [0, 1] or N < 0.  r is the KEPT fraction ("30% cache ratio"). */
+int64_t kvzip_keep_count(double r, int64_t N);
+
+/* Bytes of workspace kvzip_select needs. */
+size_t kvzip_select_workspace_size(int64_t N, int64_t n_heads);
+
+/*
+ * Keep the k largest of the N = n_heads * n_c scores (flat index
+ * f = head * n_c + j, head = l*H + h), globally across heads, so per-head
+ * budgets follow the scores (scime.ai summary, "Measured effects": uniform
+ * head budgets hurt).  Among equal scores the lower flat index is kept first,
+ * which makes the mask unique.
+ *
+ *   scores    [N] float32, finite and >= 0 (NaN/Inf give an unspecified but
+ *             in-bounds result).
+ *   k         0..N (use kvzip_keep_count for a ratio).
+ *   n_heads   >= 1, N % n_heads == 0.
+ *   keep      [N] uint8 out: 1 = kept.  Any alignment.
+ *   offsets   [n_heads + 1] int64 out: offsets[h] = kept rows in heads < h;
+ *             offsets[n_heads] = k.  8-byte aligned.
+ *   threshold float out or NULL: the k-th largest score (+inf if k == 0).
+ *   N < 2^31.
+ */
+kvzip_status kvzip_select(const float* scores, int64_t N, int64_t k, int64_t n_heads,
+                          uint8_t* keep, int64_t* offsets, float* threshold,
+                          void* workspace, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------- compaction */
+
+/* Bytes of workspace kvzip_compact needs. */
+size_t kvzip_compact_workspace_size(int64_t n_heads, int n_c);
+
+/*
+ * Pack the kept rows of K and V into per-head variable-length caches (blog
+ * post 4.1, step 5; rebuttal's decoding table: cache size scales with the
+ * kept ratio).  For each head, kept positions ascending:
+ *   k_out[offsets[h] + t] = k[h][j_t], v_out[...] = v[h][j_t], pos_out[...] = j_t.
+ *
+ *   k, v      [n_heads][n_c][d] bf16 (rows are copied bit-exactly).
+ *   keep      [n_heads * n_c] uint8 (nonzero = kept); offsets as from kvzip_select.
+ *   k_out, v_out  [offsets[n_heads]][d] bf16 out; both may be NULL only when
+ *             offsets[n_heads] == 0 (nothing kept; nothing is written then).
+ *   pos_out   [offsets[n_heads]] int32 out, or NULL.  4-byte aligned.
+ *   d         128 or 256.
+ */
+kvzip_status kvzip_compact(const void* k, const void* v, const uint8_t* keep,
+                           const int64_t* offsets, int64_t n_heads, int n_c, int d,
+                           void* k_out, void* v_out, int32_t* pos_out, void* workspace,
+                           size_t ws_bytes, void* stream);
+
+/* Number of kernel launches the most recent accepted call enqueued
+ * (process-wide; for tests and launch accounting). */
+int kvzip_last_launch_count(void);
+
+/* Static, human-readable name of a status code. */
+const char* kvzip_status_string(kvzip_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVZIP_H_ */

@@ -1,0 +1,144 @@
+"""Host-only checks of the C ABI: the library loads, exports every function
+include/kvzip.h declares, and rejects bad arguments before touching the GPU."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kvzip.h")
+
+
+@pytest.fixture(scope="module")
+def kz():
+    from attention_score_reduction_b200 import build
+    build.build()
+    from attention_score_reduction_b200 import kvzip
+    return kvzip
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvzip_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("kvzip_score_chunk", "kvzip_select", "kvzip_compact",
+                     "kvzip_score_workspace_size", "kvzip_select_workspace_size",
+                     "kvzip_compact_workspace_size", "kvzip_keep_count", "kvzip_status_string",
+                     "kvzip_workspace_status", "kvzip_set_wait_timeout_ns"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(kz):
+    lib = ctypes.CDLL(kz.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(kz):
+    for s in range(5):
+        assert kz.status_string(s)
+    assert kz.status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("r,N", [(0.3, 2048), (0.3, 4194304), (0.3, 33554432), (0.5, 33554432),
+                                 (0.25, 47185920), (0.3, 66846720), (0.0, 10), (1.0, 10),
+                                 (0.1, 10), (0.7, 123457)])
+def test_keep_count_matches_oracle(kz, r, N):
+    assert kz.keep_count(r, N) == oracle.keep_count(r, N)
+
+
+def test_keep_count_rejects(kz):
+    lib = kz.library()
+    assert lib.kvzip_keep_count(-0.1, 10) == -1
+    assert lib.kvzip_keep_count(1.5, 10) == -1
+    assert lib.kvzip_keep_count(float("nan"), 10) == -1
+    assert lib.kvzip_keep_count(0.5, -1) == -1
+
+
+def test_workspace_sizes(kz):
+    assert kz.score_workspace_size(256, 4, 2064) == 256 + 256 * (math.ceil(8256 / 256) * 256) * 4
+    assert kz.select_workspace_size(33554432, 256) > 0
+    assert kz.compact_workspace_size(256, 131072) > 0
+
+
+FAKE = 1 << 20  # a well-aligned non-null address; never dereferenced on rejected calls
+
+
+def _score(kz, **over):
+    a = dict(dt=0, q=FAKE, k=FAKE, ks=FAKE, s=FAKE, B=2, G=4, n_in=100, n_c=1000, d=128,
+             scale=0.0, ws=FAKE, ws_bytes=1 << 30, stream=None)
+    a.update(over)
+    return kz.library().kvzip_score_chunk(a["dt"], a["q"], a["k"], a["ks"], a["s"], a["B"], a["G"],
+                                          a["n_in"], a["n_c"], a["d"], a["scale"], a["ws"],
+                                          a["ws_bytes"], a["stream"])
+
+
+def test_score_rejects_bad_arguments(kz):
+    assert _score(kz, dt=7) == kz.ERR_INVALID_ARG
+    assert _score(kz, q=None) == kz.ERR_INVALID_ARG
+    assert _score(kz, k=None) == kz.ERR_INVALID_ARG
+    assert _score(kz, ks=None) == kz.ERR_INVALID_ARG
+    assert _score(kz, s=None) == kz.ERR_INVALID_ARG
+    assert _score(kz, ws=None) == kz.ERR_INVALID_ARG
+    assert _score(kz, d=64) == kz.ERR_UNSUPPORTED
+    assert _score(kz, d=0) == kz.ERR_INVALID_ARG
+    assert _score(kz, B=-1) == kz.ERR_INVALID_ARG
+    assert _score(kz, q=FAKE + 8) == kz.ERR_INVALID_ARG        # not 16-byte aligned
+    assert _score(kz, s=FAKE + 2) == kz.ERR_INVALID_ARG        # not 4-byte aligned
+    assert _score(kz, ws=FAKE + 16) == kz.ERR_INVALID_ARG      # not 256-byte aligned
+    assert _score(kz, ws_bytes=100) == kz.ERR_INVALID_ARG
+    assert _score(kz, B=70000) == kz.ERR_UNSUPPORTED
+
+
+def test_score_empty_is_noop(kz):
+    for over in (dict(B=0), dict(G=0), dict(n_in=0), dict(n_c=0)):
+        assert _score(kz, q=None, k=None, ks=None, s=None, ws=None, **over) == kz.OK
+
+
+def _select(kz, **over):
+    a = dict(s=FAKE, N=1000, k=300, H=10, keep=FAKE, off=FAKE, thr=None, ws=FAKE,
+             ws_bytes=1 << 30)
+    a.update(over)
+    return kz.library().kvzip_select(a["s"], a["N"], a["k"], a["H"], a["keep"], a["off"], a["thr"],
+                                     a["ws"], a["ws_bytes"], None)
+
+
+def test_select_rejects_bad_arguments(kz):
+    assert _select(kz, k=1001) == kz.ERR_INVALID_ARG
+    assert _select(kz, k=-1) == kz.ERR_INVALID_ARG
+    assert _select(kz, H=0) == kz.ERR_INVALID_ARG
+    assert _select(kz, H=7) == kz.ERR_INVALID_ARG              # 1000 % 7 != 0
+    assert _select(kz, s=None) == kz.ERR_INVALID_ARG
+    assert _select(kz, keep=None) == kz.ERR_INVALID_ARG
+    assert _select(kz, off=None) == kz.ERR_INVALID_ARG
+    assert _select(kz, s=FAKE + 4) == kz.ERR_INVALID_ARG       # scores need 16-byte alignment
+    assert _select(kz, off=FAKE + 4) == kz.ERR_INVALID_ARG
+    assert _select(kz, ws_bytes=10) == kz.ERR_INVALID_ARG
+    assert _select(kz, N=1 << 31, k=0, H=1) == kz.ERR_INVALID_ARG
+
+
+def _compact(kz, **over):
+    a = dict(k=FAKE, v=FAKE, keep=FAKE, off=FAKE, H=4, n_c=100, d=128, ko=FAKE, vo=FAKE, pos=None,
+             ws=FAKE, ws_bytes=1 << 30)
+    a.update(over)
+    return kz.library().kvzip_compact(a["k"], a["v"], a["keep"], a["off"], a["H"], a["n_c"], a["d"],
+                                      a["ko"], a["vo"], a["pos"], a["ws"], a["ws_bytes"], None)
+
+
+def test_compact_rejects_bad_arguments(kz):
+    assert _compact(kz, d=64) == kz.ERR_UNSUPPORTED
+    assert _compact(kz, H=0) == kz.ERR_INVALID_ARG
+    assert _compact(kz, k=None) == kz.ERR_INVALID_ARG
+    assert _compact(kz, vo=None) == kz.ERR_INVALID_ARG
+    assert _compact(kz, k=FAKE + 8) == kz.ERR_INVALID_ARG
+    assert _compact(kz, pos=FAKE + 2) == kz.ERR_INVALID_ARG
+    assert _compact(kz, ws_bytes=1) == kz.ERR_INVALID_ARG
+    assert _compact(kz, n_c=0, k=None) == kz.OK

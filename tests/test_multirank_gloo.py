@@ -1,0 +1,66 @@
+"""Host logic of multi-GPU runs, on CPU with gloo and two ranks: each rank
+compresses its own context (distinct seeds), and the reported time is the
+max over ranks."""
+import os
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from attention_score_reduction_b200 import benchutil as bu
+        from attention_score_reduction_b200 import synth
+        r, w, lr = bu.dist_env()
+        assert (r, w, lr) == (rank, world, rank)
+        wl = synth.WORKLOADS["tiny_fp32"]
+        if r:
+            wl = wl.with_(cfg_id=wl.cfg_id + bu.rank_salt(r))
+        k = synth.context_keys(wl)
+        digest = float(k.double().sum())
+        got = bu.max_over_ranks(10.0 + rank, world)
+        allk = [None] * world
+        dist.all_gather_object(allk, digest)
+        bu.barrier(world)
+        q.put((rank, got, allk))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_max_time_and_distinct_contexts():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29500 + (os.getpid() % 1000)
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, got, allk in res:
+        assert got == 11.0                       # max over ranks of 10 + rank
+        assert allk[0] != allk[1]                # each rank has its own context
+
+
+def test_clock_summary_parsing():
+    from attention_score_reduction_b200 import benchutil as bu
+    rows = [["0", "1965", "1965", "700.1", "0x0", "Not Active", "Not Active", "Not Active", "Not Active"],
+            ["0", "1800", "1965", "990.0", "0x4", "Not Active", "Not Active", "Not Active", "Active"],
+            ["0", "1700", "1965", "1000.0", "0x4", "Not Active", "Not Active", "Not Active", "Active"]]
+    s = bu.summarize_clock_rows(rows)
+    assert s["sm_mhz"] == 1800 and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"]
+
+
+def test_score_flops_counts_pairs():
+    from attention_score_reduction_b200 import benchutil as bu
+    f = bu.score_flops(B=2, G=3, n_in=5, n_c=7, d=4)
+    R = 15
+    assert f["pass2"] == 2 * 4 * 2 * R * 7
+    assert f["pass1"] == 2 * 4 * 2 * (R * 7 + 3 * 5 * 6 // 2)
