@@ -19,7 +19,9 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
+#include "kvzip.h"
 #include "kvzip_internal.h"
 
 namespace kvzip {
@@ -365,3 +367,78 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launches) {
 }
 
 }  // namespace kvzip
+
+// ---------------------------------------------------------------------------
+// Allocation-free selection: kvzip_select_noalloc.
+//
+// Some callers cannot hand the library a workspace: code that runs inside a
+// host process whose device memory is owned by someone else's pool (a plugin
+// in a serving engine that has reserved the GPU's memory up front), or a
+// latency-critical loop that may not call cudaMalloc because it can block and
+// synchronise the device.  For them the selection scratch lives in this
+// file-scope array instead; every GPU that loads the library holds it until
+// the process exits.  Its contents survive between calls: the selection
+// kernels re-initialise the state and histograms at the start of every call,
+// and every per-block count is written before it is read.  All calls on one
+// device share the array, so calls that overlap on the GPU (different
+// streams, no ordering) race and give wrong masks.
+namespace kvzip {
+namespace {
+
+constexpr size_t kSelectStaticBytes = size_t{1} << 20;  // 1 MiB
+__device__ __align__(256) uint8_t g_select_scratch[kSelectStaticBytes];
+
+constexpr int kMaxDevices = 64;
+void* g_scratch_ptr[kMaxDevices] = {};
+std::mutex g_scratch_mu;
+
+// Device address of g_select_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device (with that device current) and cached.
+cudaError_t static_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_select_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace kvzip
+
+extern "C" kvzip_status kvzip_select_noalloc(const float* scores, int64_t N, int64_t k,
+                                             int64_t n_heads, uint8_t* keep, int64_t* offsets,
+                                             float* threshold, void* stream) {
+  if (N <= 0 || n_heads <= 0 || k < 0 || k > N) return KVZIP_ERR_INVALID_ARG;
+  if (N % n_heads != 0 || N >= (int64_t{1} << 31)) return KVZIP_ERR_INVALID_ARG;
+  if (!scores || !keep || !offsets) return KVZIP_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(scores) & 15) || (reinterpret_cast<uintptr_t>(offsets) & 7) ||
+      (threshold && (reinterpret_cast<uintptr_t>(threshold) & 3)))
+    return KVZIP_ERR_INVALID_ARG;
+  // Larger problems need more scratch than the static array holds.
+  if (kvzip::select_ws_bytes(N, n_heads) > kvzip::kSelectStaticBytes) return KVZIP_ERR_UNSUPPORTED;
+  void* ws = nullptr;
+  if (kvzip::static_scratch(&ws) != cudaSuccess) return KVZIP_ERR_CUDA;
+  kvzip::SelectArgs a;
+  a.scores = scores;
+  a.N = N;
+  a.k = k;
+  a.n_heads = n_heads;
+  a.n_c = N / n_heads;
+  a.keep = keep;
+  a.offsets = offsets;
+  a.threshold = threshold;
+  a.ws = ws;
+  a.ws_bytes = kvzip::kSelectStaticBytes;
+  int launches = 0;
+  const cudaError_t e = kvzip::launch_select(a, static_cast<cudaStream_t>(stream), &launches);
+  return e == cudaSuccess ? KVZIP_OK : KVZIP_ERR_CUDA;
+}

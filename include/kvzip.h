@@ -146,6 +146,31 @@ kvzip_status kvzip_select(const float* scores, int64_t N, int64_t k, int64_t n_h
                           uint8_t* keep, int64_t* offsets, float* threshold,
                           void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * kvzip_select without a workspace, for callers that cannot allocate device
+ * memory: e.g. a plugin inside a serving engine whose memory pool has already
+ * claimed the GPU, or a latency-critical loop where cudaMalloc (which can
+ * block and synchronise the device) is not allowed.  The pages have no
+ * counterpart to this; it is a deployment convenience.
+ *
+ * Same arguments and results as kvzip_select, but the selection scratch is a
+ * library-owned static device array of 1 MiB on every GPU that loads the
+ * library (held until the process exits).  It fits problems with
+ * kvzip_select_workspace_size(N, n_heads) <= 1 MiB, i.e. roughly
+ * n_heads * ceil(n_c / 8192) <= 128000 (all LLaMA3.1-8B / Qwen2.5-14B /
+ * Gemma3-12B shapes up to 170K tokens); larger ones return
+ * KVZIP_ERR_UNSUPPORTED without launching anything.  N must be >= 1.
+ *   - The first call on each device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - All calls on a device share the array: calls that overlap on the GPU
+ *     (e.g. on unordered streams) race.  The array keeps the last call's
+ *     contents; each call re-initialises what must start at zero.
+ *   - Allocates nothing (no cudaMalloc / cudaFree, no allocating library call).
+ */
+kvzip_status kvzip_select_noalloc(const float* scores, int64_t N, int64_t k, int64_t n_heads,
+                                  uint8_t* keep, int64_t* offsets, float* threshold,
+                                  void* stream);
+
 /* --------------------------------------------------------------- compaction */
 
 /* Bytes of workspace kvzip_compact needs. */
