@@ -15,6 +15,7 @@ namespace {
 
 std::atomic<uint64_t> g_timeout_ns{2000000000ull};
 std::atomic<int> g_last_launches{0};
+std::atomic<int> g_test_stall{0};
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -40,6 +41,8 @@ const char* kvzip_status_string(kvzip_status s) {
 void kvzip_set_wait_timeout_ns(uint64_t ns) {
   g_timeout_ns.store(ns == 0 ? 2000000000ull : ns);
 }
+
+void kvzip_set_test_stall(int on) { g_test_stall.store(on ? 1 : 0); }
 
 /* Number of kernel launches the most recent successful call enqueued (testing aid). */
 int kvzip_last_launch_count(void) { return g_last_launches.load(); }
@@ -84,6 +87,7 @@ static kvzip_status score_passes(int passes, kvzip_dtype dt, const void* q, cons
   a.scale = scale;
   a.timeout_ns = g_timeout_ns.load();
   a.passes = passes;
+  a.test_stall = g_test_stall.load();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int launches = 0;
   cudaError_t e = (dt == KVZIP_BF16) ? kvzip::launch_score_tc(a, s, &launches)
@@ -211,6 +215,19 @@ kvzip_status kvzip_compact(const void* k, const void* v, const uint8_t* keep,
   a.ws_bytes = ws_bytes;
   int launches = 0;
   cudaError_t e = kvzip::launch_compact(a, static_cast<cudaStream_t>(stream), &launches);
+  if (e == cudaSuccess) g_last_launches.store(launches);
+  return from_cuda(e);
+}
+
+kvzip_status kvzip_head_scores(const float* scores, int64_t n_heads, int64_t n_c,
+                               float* head_scores, void* stream) {
+  if (n_heads <= 0 || n_c <= 0 || n_heads > (int64_t{1} << 24) || n_c >= (int64_t{1} << 31))
+    return KVZIP_ERR_INVALID_ARG;
+  if (!scores || !head_scores || !aligned(scores, 4) || !aligned(head_scores, 4))
+    return KVZIP_ERR_INVALID_ARG;
+  int launches = 0;
+  cudaError_t e = kvzip::launch_head_scores(scores, n_heads, n_c, head_scores,
+                                            static_cast<cudaStream_t>(stream), &launches);
   if (e == cudaSuccess) g_last_launches.store(launches);
   return from_cuda(e);
 }

@@ -28,6 +28,7 @@ struct ScoreArgs {
   float scale;
   uint64_t timeout_ns;
   int passes;         // bit 0: pass 1 (row log-sum-exp), bit 1: pass 2 (column max)
+  int test_stall;     // tensor-core scorer only: loader issues nothing (timeout tests)
 };
 
 // Tensor-core (tcgen05) scorer for bf16 inputs.  Returns a cudaError_t.
@@ -62,5 +63,9 @@ struct CompactArgs {
 };
 size_t compact_ws_bytes(int64_t n_heads, int n_c);
 cudaError_t launch_compact(const CompactArgs& a, cudaStream_t s, int* launches);
+
+// Head-level scores: out[h] = max_j scores[h][j].
+cudaError_t launch_head_scores(const float* scores, int64_t n_heads, int64_t n_c, float* out,
+                               cudaStream_t s, int* launches);
 
 }  // namespace kvzip

@@ -49,6 +49,13 @@ constexpr int kThreads = 320;        // 10 warps
 constexpr int kBM = 128;             // rows per A tile (M of the MMA)
 constexpr int kATiles = 2;           // A tiles per CTA
 constexpr uint64_t kDrainTimeoutNs = 1000000000ull;
+// Pass 1: out of every 8 pairs of exponentials, this many are evaluated by
+// polynomial on the FMA pipe instead of the MUFU unit (16 ex2 per clock per SM,
+// half the tensor core's 32 logits per clock at d = 128).
+#ifndef KVZIP_POLY_PAIRS
+#define KVZIP_POLY_PAIRS 0
+#endif
+constexpr int kPolyPairs = KVZIP_POLY_PAIRS;
 
 template <int D>
 struct TcLayout {
@@ -61,9 +68,11 @@ struct TcLayout {
   static constexpr int B_BYTES = KB * B_KB_BYTES;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + kATiles * A_BYTES;
-  static constexpr int OFF_BAR = OFF_B + STAGES * B_BYTES;
-  // barriers: a_full, b_full[S], b_empty[S], s_full[2][2], s_empty[2][2], mma_done
-  static constexpr int N_BARS = 1 + 2 * STAGES + 8 + 1;
+  static constexpr int L_BYTES = BN * 4;                // pass 2: lse2 of one B tile
+  static constexpr int OFF_L = OFF_B + STAGES * B_BYTES;
+  static constexpr int OFF_BAR = OFF_L + STAGES * L_BYTES;
+  // barriers: a_full, b_full[S], b_empty[S], s_full[2][2], s_empty[2][2], mma_done, l_empty[S]
+  static constexpr int N_BARS = 1 + 2 * STAGES + 8 + 1 + STAGES;
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;  // tmem base, abort flag
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = BYTES + 1024;        // slack for 1024-B alignment
@@ -133,6 +142,10 @@ __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, uint3
   }
 }
 
+// The whole BN-column accumulator row of this thread in one TMEM round trip.
+__device__ __forceinline__ void tmem_ld_tile(uint32_t taddr, float (&v)[128]) { tmem_ld128(taddr, v); }
+__device__ __forceinline__ void tmem_ld_tile(uint32_t taddr, float (&v)[64]) { tmem_ld64(taddr, v); }
+
 struct TcParams {
   float* scores;
   float* lse2;
@@ -140,6 +153,7 @@ struct TcParams {
   int G, n_in, n_c, R, R_pad;
   float c;            // scale * log2(e)
   uint64_t timeout_ns;
+  int test_stall;     // test hook: the loader issues no copies, so every wait runs out
 };
 
 template <int D, bool PASS2>
@@ -162,6 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_full = bars + 1 + 2 * STAGES;        // [t*2 + buf]
   uint64_t* s_empty = bars + 1 + 2 * STAGES + 4;   // [t*2 + buf]
   uint64_t* mma_done = bars + 1 + 2 * STAGES + 8;
+  uint64_t* l_empty = bars + 2 + 2 * STAGES + 8;    // pass 2: lse2 stage free again
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::OFF_MISC + 4);
 
@@ -194,6 +209,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s_empty[i], kBM);
     }
     mbar_init(mma_done, 1);
+    // every thread of every active epilogue group releases each lse2 stage
+    for (int s = 0; s < STAGES; ++s) mbar_init(&l_empty[s], nA * kBM);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -213,18 +230,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&amap);
       tma_prefetch_desc(&bmap0);
       if (!PASS2) tma_prefetch_desc(&bmap1);
-      mbar_arrive_expect_tx(a_full, nA * Lay::A_BYTES);
-      for (int t = 0; t < nA; ++t)
-        for (int kb = 0; kb < KB; ++kb)
-          tma_load_3d(smem + Lay::OFF_A + t * Lay::A_BYTES + kb * Lay::A_KB_BYTES, &amap, a_full,
-                      kb * 64, a_row0 + t * kBM, b);
+      const bool stall = p.test_stall != 0;
+      if (!stall) {
+        mbar_arrive_expect_tx(a_full, nA * Lay::A_BYTES);
+        for (int t = 0; t < nA; ++t)
+          for (int kb = 0; kb < KB; ++kb)
+            tma_load_3d(smem + Lay::OFF_A + t * Lay::A_BYTES + kb * Lay::A_KB_BYTES, &amap,
+                        a_full, kb * 64, a_row0 + t * kBM, b);
+      }
       int issued = 0;
 #pragma unroll 1
-      for (int it = 0; it < n_b; ++it) {
+      for (int it = 0; !stall && it < n_b; ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         if (!wait_one(&b_empty[s], ph ^ 1, ctl)) break;
-        mbar_arrive_expect_tx(&b_full[s], Lay::B_BYTES);
+        if (PASS2 && !wait_one(&l_empty[s], ph ^ 1, ctl)) break;
+        mbar_arrive_expect_tx(&b_full[s], Lay::B_BYTES + (PASS2 ? Lay::L_BYTES : 0));
         const void* map = &bmap0;
         int row = it * BN;
         if (!PASS2 && it >= n_kt_ctx) {
@@ -234,10 +255,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* dst = smem + Lay::OFF_B + s * Lay::B_BYTES;
         for (int kb = 0; kb < KB; ++kb)
           tma_load_3d(dst + kb * Lay::B_KB_BYTES, map, &b_full[s], kb * 64, row, b);
+        if (PASS2)  // the row normalisers of this query tile ride on the same barrier
+          bulk_load(smem + Lay::OFF_L + s * Lay::L_BYTES,
+                    p.lse2 + static_cast<size_t>(b) * p.R_pad + row, Lay::L_BYTES, &b_full[s]);
         issued = it + 1;
       }
       // Drain: every copy this CTA started must land before shared memory is released.
-      wait_drain(a_full, 0, p.status);
+      if (!stall) wait_drain(a_full, 0, p.status);
       for (int s = 0; s < STAGES && s < issued; ++s) {
         const int last = s + ((issued - 1 - s) / STAGES) * STAGES;
         wait_drain(&b_full[s], (last / STAGES) & 1, p.status);
@@ -304,9 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float v[BN];
           const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                  (t * 2 + buf) * BN;
-#pragma unroll
-          for (int c0 = 0; c0 < BN; c0 += 32)
-            tmem_ld32(taddr + c0, *reinterpret_cast<float(*)[32]>(&v[c0]));
+          tmem_ld_tile(taddr, v);
           tc_fence_before();
           mbar_arrive(&s_empty[t * 2 + buf]);
           // masks: ragged context tail, causal self keys
@@ -332,15 +354,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           mx0 = fmax3(mx0, mx1, fmaxf(v[BN - 2], v[BN - 1]));
           const float m_new = fmaxf(m, mx0 * c);
           const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+          // x = c*s - m in packed pairs; of every 8 pairs, kPolyPairs take 2^x on
+          // the FMA pipe and the rest on the MUFU unit, so both pipes share the work.
+          const float2 c2 = make_float2(c, c);
+          const float2 nm2 = make_float2(-m_use, -m_use);
+          float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int j = 0; j < BN; j += 4) {
-            a0 += ex2_approx(fmaf(v[j + 0], c, -m_use));
-            a1 += ex2_approx(fmaf(v[j + 1], c, -m_use));
-            a2 += ex2_approx(fmaf(v[j + 2], c, -m_use));
-            a3 += ex2_approx(fmaf(v[j + 3], c, -m_use));
+          for (int j = 0; j < BN; j += 16) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float2 x = ffma2(make_float2(v[j + 2 * q], v[j + 2 * q + 1]), c2, nm2);
+              float2 e;
+              if (q < kPolyPairs) {
+                e = exp2_poly2(x);
+              } else {
+                e.x = ex2_approx(x.x);
+                e.y = ex2_approx(x.y);
+              }
+              if (q & 1)
+                acc1 = fadd2(acc1, e);
+              else
+                acc0 = fadd2(acc0, e);
+            }
           }
-          l = fmaf(l, ex2_approx(m - m_use), (a0 + a1) + (a2 + a3));
+          l = fmaf(l, ex2_approx(m - m_use), (acc0.x + acc0.y) + (acc1.x + acc1.y));
           m = m_new;
         }
         if (!*abort_flag && arow < p.R_pad)
@@ -348,30 +385,32 @@ __global__ void __launch_bounds__(kThreads, 1)
               (arow < p.R) ? m + lg2_approx(l) : INFINITY;
       } else {
         // ---------------- pass 2: running max over query rows of c*s - lse2
-        const float* lse_row = p.lse2 + static_cast<size_t>(b) * p.R_pad;
         float best = -INFINITY;
 #pragma unroll 1
         for (int it = 0; it < n_b; ++it) {
           const int buf = it & 1;
+          const int st = it % STAGES;
+          // The stage's lse2 bytes landed with b_full; the stage cannot be refilled
+          // before this group releases l_empty, so this phase is still the latest.
+          if (!wait_warp(&b_full[st], (it / STAGES) & 1, ctl)) break;
           if (!wait_warp(&s_full[t * 2 + buf], (it >> 1) & 1, ctl)) break;
           tc_fence_after();
           float v[BN];
           const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                  (t * 2 + buf) * BN;
-#pragma unroll
-          for (int c0 = 0; c0 < BN; c0 += 32)
-            tmem_ld32(taddr + c0, *reinterpret_cast<float(*)[32]>(&v[c0]));
+          tmem_ld_tile(taddr, v);
           tc_fence_before();
           mbar_arrive(&s_empty[t * 2 + buf]);
-          const float4* L4 = reinterpret_cast<const float4*>(lse_row + it * BN);
+          const float4* L4 = reinterpret_cast<const float4*>(smem + Lay::OFF_L + st * Lay::L_BYTES);
           float b0 = best, b1 = -INFINITY;
 #pragma unroll
           for (int j = 0; j < BN; j += 4) {
-            const float4 L = __ldg(L4 + j / 4);
+            const float4 L = L4[j / 4];   // same address in every lane: broadcast
             b0 = fmax3(b0, fmaf(v[j + 0], c, -L.x), fmaf(v[j + 1], c, -L.y));
             b1 = fmax3(b1, fmaf(v[j + 2], c, -L.z), fmaf(v[j + 3], c, -L.w));
           }
           best = fmaxf(b0, b1);
+          mbar_arrive(&l_empty[st]);
         }
         if (!*abort_flag && arow < p.n_c) {
           float* dst = p.scores + static_cast<size_t>(b) * p.n_c + arow;
@@ -456,6 +495,7 @@ static cudaError_t launch_tc(const ScoreArgs& a, cudaStream_t s, int* launches) 
   p.R_pad = a.R_pad;
   p.c = a.scale * 1.4426950408889634f;
   p.timeout_ns = a.timeout_ns;
+  p.test_stall = a.test_stall;
 
   if (a.passes & 1) {
     dim3 g1((a.R + kATiles * kBM - 1) / (kATiles * kBM), a.B);

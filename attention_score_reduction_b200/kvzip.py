@@ -40,11 +40,13 @@ def _load() -> ctypes.CDLL:
         "kvzip_score_colmax": (i32, [i32, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, sz, vp]),
         "kvzip_workspace_status": (i32, [vp, vp]),
         "kvzip_set_wait_timeout_ns": (None, [u64]),
+        "kvzip_set_test_stall": (None, [i32]),
         "kvzip_keep_count": (i64, [f64, i64]),
         "kvzip_select_workspace_size": (sz, [i64, i64]),
         "kvzip_select": (i32, [vp, i64, i64, i64, vp, vp, vp, vp, sz, vp]),
         "kvzip_compact_workspace_size": (sz, [i64, i32]),
         "kvzip_compact": (i32, [vp, vp, vp, vp, i64, i32, i32, vp, vp, vp, vp, sz, vp]),
+        "kvzip_head_scores": (i32, [vp, i64, i64, vp, vp]),
         "kvzip_last_launch_count": (i32, []),
         "kvzip_status_string": (ctypes.c_char_p, [i32]),
     }
@@ -146,6 +148,11 @@ def set_wait_timeout_ns(ns: int):
     _lib.kvzip_set_wait_timeout_ns(int(ns))
 
 
+def set_test_stall(on: bool):
+    """Timeout-path test hook: the scoring loader issues no copies while on."""
+    _lib.kvzip_set_test_stall(1 if on else 0)
+
+
 def read_lse(workspace: torch.Tensor, B: int, G: int, n_in: int) -> torch.Tensor:
     """Natural-log row normalisers the last pass-1 launch left in the workspace,
     [B][G*n_in] (a view into the workspace's padded buffer, converted)."""
@@ -220,6 +227,18 @@ def compact(k: torch.Tensor, v: torch.Tensor, keep: torch.Tensor, offsets: torch
                            workspace.numel(), _stream(stream))
     _check(s, "kvzip_compact")
     return k_out, v_out, pos_out
+
+
+# ---------------------------------------------------------------- head scores
+
+def head_scores(scores: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+    """max over positions of each head's scores; scores [n_heads][n_c] float32."""
+    _dev_contig("scores", scores, torch.float32)
+    n_heads, n_c = scores.shape
+    out = torch.empty(n_heads, dtype=torch.float32, device=scores.device) if out is None else out
+    _check(_lib.kvzip_head_scores(_ptr(scores), n_heads, n_c, _ptr(out), _stream(stream)),
+           "kvzip_head_scores")
+    return out
 
 
 def last_launch_count() -> int:

@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--workload", default="llama8b_128k", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--r", type=float, default=None, help="kept fraction (default: first of workload)")
     ap.add_argument("--chunk", type=int, default=None, help="override context rows per chunk")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="override the layer count (smaller cases for profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--e2e-steps", type=int, default=None)
@@ -54,6 +56,8 @@ def workload(args, rank=0):
     wl = synth.WORKLOADS[args.workload]
     if args.chunk:
         wl = wl.with_(m=args.chunk)
+    if args.layers:
+        wl = wl.with_(L=args.layers)
     if rank:
         wl = wl.with_(cfg_id=wl.cfg_id + bu.rank_salt(rank))
     return wl

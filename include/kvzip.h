@@ -116,6 +116,13 @@ kvzip_status kvzip_workspace_status(void* workspace, void* stream);
  * default.  Intended for tests of the timeout path. */
 void kvzip_set_wait_timeout_ns(uint64_t ns);
 
+/* Test hook for the timeout path: while on (nonzero), the bf16 scoring
+ * kernels' loader warp issues no copies, so every pipeline wait in them runs
+ * out after the wait timeout and the call reports KVZIP_ERR_TIMEOUT through
+ * kvzip_workspace_status.  Nothing faults or hangs.  Process-wide; applies to
+ * launches enqueued after the call.  Leave off in normal use. */
+void kvzip_set_test_stall(int on);
+
 /* ---------------------------------------------------------------- selection */
 
 /* k = ceil(r * N), the product taken in IEEE double; -1 if r is outside
@@ -193,6 +200,19 @@ kvzip_status kvzip_compact(const void* k, const void* v, const uint8_t* keep,
                            const int64_t* offsets, int64_t n_heads, int n_c, int d,
                            void* k_out, void* v_out, int32_t* pos_out, void* workspace,
                            size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------ head scores */
+
+/*
+ * Head-level importance, head_scores[h] = max_j scores[h][j] over the n_c
+ * positions of each of the n_heads = L*H heads (OpenReview rebuttal, answer on
+ * how the head-level scores for the DuoAttention comparison were computed:
+ * max over the sequence dimension of the L x H x n_c score tensor).  Exact.
+ *   scores       [n_heads][n_c] float32, finite and >= 0; 4-byte aligned.
+ *   head_scores  [n_heads] float32 out; 4-byte aligned.
+ */
+kvzip_status kvzip_head_scores(const float* scores, int64_t n_heads, int64_t n_c,
+                               float* head_scores, void* stream);
 
 /* Number of kernel launches the most recent accepted call enqueued
  * (process-wide; for tests and launch accounting). */

@@ -142,3 +142,11 @@ def test_compact_rejects_bad_arguments(kz):
     assert _compact(kz, pos=FAKE + 2) == kz.ERR_INVALID_ARG
     assert _compact(kz, ws_bytes=1) == kz.ERR_INVALID_ARG
     assert _compact(kz, n_c=0, k=None) == kz.OK
+
+
+def test_head_scores_rejects_bad_arguments(kz):
+    lib = kz.library()
+    assert lib.kvzip_head_scores(None, 4, 10, FAKE, None) == kz.ERR_INVALID_ARG
+    assert lib.kvzip_head_scores(FAKE, 0, 10, FAKE, None) == kz.ERR_INVALID_ARG
+    assert lib.kvzip_head_scores(FAKE, 4, 0, FAKE, None) == kz.ERR_INVALID_ARG
+    assert lib.kvzip_head_scores(FAKE + 2, 4, 10, FAKE, None) == kz.ERR_INVALID_ARG

@@ -223,3 +223,15 @@ def test_small_context_end_to_end(kz):
     assert np.array_equal(ko.cpu().view(torch.int16).numpy(), ko_ref)
     assert np.array_equal(vo.cpu().view(torch.int16).numpy(), vo_ref)
     assert np.array_equal(pos.cpu().numpy(), pos_ref)
+
+
+# ------------------------------------------------------------------ head scores
+
+@pytest.mark.parametrize("n_heads,n_c", [(256, 16384), (3, 40000), (5, 7), (1, 1)])
+def test_head_scores_bit_exact(kz, n_heads, n_c):
+    from attention_score_reduction_b200 import synth
+    s = synth.random_scores(n_heads, n_c, seed=n_heads + n_c)
+    got = kz.head_scores(s.cuda()).cpu().numpy()
+    L = 1
+    want = oracle.head_scores(s.numpy(), L, n_heads)[0]
+    assert np.array_equal(got, want.astype(np.float32))
