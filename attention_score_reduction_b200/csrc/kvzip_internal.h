@@ -13,8 +13,10 @@ constexpr uint32_t kStatusTimeout = 1u;
 // Bytes reserved at the front of the scoring workspace for the status word.
 constexpr size_t kScoreWsHeader = 256;
 
-// Query rows of one unit are padded to this many in the log-sum-exp buffer.
-constexpr int kRowPad = 256;
+// Query rows of one unit are padded to a multiple of this many in the
+// log-sum-exp buffer (a multiple of the pass-1 CTA's 256 rows and of every
+// pass-2 query tile height: 96 and 64).
+constexpr int kRowPad = 768;
 
 struct ScoreArgs {
   const void* q;

@@ -15,10 +15,26 @@
 //   c * s - lse2[rho]; exp is monotone, so one exp2 per key at the end:
 //   p_j = 2^(max_rho (c s_rho,j - lse2[rho])).
 //
-// One skeleton serves both passes: warp 0 issues TMA loads (A tiles once, then
-// a STAGES-deep ring of B tiles), warp 1 allocates TMEM and issues tcgen05.mma
-// from one thread, warps 2..9 are two 128-thread epilogue groups, one per A
-// tile, each reading its own double-buffered fp32 accumulator from TMEM.
+// One skeleton serves both passes.  The A tile of a CTA never changes, so it
+// lives in tensor memory: each epilogue thread copies its own row there once
+// (tcgen05.st), and every MMA reads A from TMEM and only B from shared memory
+// (tcgen05.mma with A in TMEM).  That halves the shared-memory operand traffic
+// per MMA, which otherwise limits a 128 x N x 16 MMA with both operands in
+// shared memory to about half the tensor core's rate on B200.
+//   warp 0      : TMA producer, a STAGES-deep ring of B tiles (+ pass-2 lse2 tiles)
+//   warps 1, 2  : one MMA-issuing thread each, for A tile 0 and A tile 1 (warp 1
+//                 also allocates TMEM).  tcgen05.mma issue stalls until the
+//                 previous MMA is nearly done, so one thread's barrier waits and
+//                 fences between batches idle the tensor pipe (measured: 113
+//                 instead of 64 cycles per 128x128x16 MMA); with two issuers one
+//                 feeds the pipe while the other waits.
+//   warps 3..18 : four 128-thread epilogue groups, one per (A tile, accumulator
+//                 buffer); the even group of each A tile first copies the A
+//                 rows into TMEM.  A group drains its BN-column accumulator in
+//                 two TMEM loads, so the tile's B tiles alternate between two
+//                 groups (four epilogue warps per scheduler: the epilogue math
+//                 is latency-bound with two).
+// TMEM map (512 columns): [0, 2*D/2) A tiles, then (tile, buffer) accumulators.
 // Every wait is bounded; on timeout the CTA records KVZIP_ERR_TIMEOUT in the
 // status word, drains its in-flight copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -36,16 +52,17 @@ template <int D>
 struct TcCfg;
 template <>
 struct TcCfg<128> {
-  static constexpr int BN = 128;     // rows per B tile (N of the MMA)
-  static constexpr int STAGES = 4;   // B ring depth
+  static constexpr int BN = 96;      // rows per B tile (N of the MMA)
+  static constexpr int STAGES = 6;   // B ring depth
 };
 template <>
 struct TcCfg<256> {
   static constexpr int BN = 64;
-  static constexpr int STAGES = 3;
+  static constexpr int STAGES = 5;
 };
 
-constexpr int kThreads = 320;        // 10 warps
+constexpr int kEpiThreads = 512;     // four 128-thread epilogue groups
+constexpr int kThreads = 32 * (1 + 2) + kEpiThreads;   // producer, 2 MMA issuers, epilogue
 constexpr int kBM = 128;             // rows per A tile (M of the MMA)
 constexpr int kATiles = 2;           // A tiles per CTA
 constexpr uint64_t kDrainTimeoutNs = 1000000000ull;
@@ -53,7 +70,7 @@ constexpr uint64_t kDrainTimeoutNs = 1000000000ull;
 // polynomial on the FMA pipe instead of the MUFU unit (16 ex2 per clock per SM,
 // half the tensor core's 32 logits per clock at d = 128).
 #ifndef KVZIP_POLY_PAIRS
-#define KVZIP_POLY_PAIRS 0
+#define KVZIP_POLY_PAIRS 2
 #endif
 constexpr int kPolyPairs = KVZIP_POLY_PAIRS;
 
@@ -62,23 +79,26 @@ struct TcLayout {
   static constexpr int BN = TcCfg<D>::BN;
   static constexpr int STAGES = TcCfg<D>::STAGES;
   static constexpr int KB = D / 64;                      // 128-byte K blocks per row
-  static constexpr int A_KB_BYTES = kBM * 128;           // one K block of an A tile
-  static constexpr int A_BYTES = KB * A_KB_BYTES;
   static constexpr int B_KB_BYTES = BN * 128;
   static constexpr int B_BYTES = KB * B_KB_BYTES;
-  static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + kATiles * A_BYTES;
-  static constexpr int L_BYTES = BN * 4;                // pass 2: lse2 of one B tile
+  static constexpr int L_BYTES = BN * 4;                 // pass 2: lse2 of one B tile
+  static constexpr int OFF_B = 0;
   static constexpr int OFF_L = OFF_B + STAGES * B_BYTES;
   static constexpr int OFF_BAR = OFF_L + STAGES * L_BYTES;
   // barriers: a_full, b_full[S], b_empty[S], s_full[2][2], s_empty[2][2], mma_done, l_empty[S]
   static constexpr int N_BARS = 1 + 2 * STAGES + 8 + 1 + STAGES;
-  static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;  // tmem base, abort flag
+  static constexpr int OFF_XCHG = OFF_BAR + 8 * N_BARS;  // parity merge, float2 per row
+  static constexpr int OFF_MISC = OFF_XCHG + kATiles * kBM * 8;  // tmem base, abort flag
   static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int CH = BN / 2;                      // accumulator columns per TMEM load
   static constexpr int SMEM_ALLOC = BYTES + 1024;        // slack for 1024-B alignment
-  static constexpr int TMEM_COLS = kATiles * 2 * BN;     // 2 buffers per A tile
-  static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of 2");
+  static constexpr int A_COLS = D / 2;                   // TMEM columns of one A tile
+  static constexpr int ACC0 = kATiles * A_COLS;          // first accumulator column
+  static constexpr int TMEM_COLS = 512;
+  static_assert(ACC0 + kATiles * 2 * BN <= TMEM_COLS, "TMEM over-committed");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "invalid MMA N");
   static_assert(SMEM_ALLOC <= 232448, "exceeds 227 KB of shared memory");
+  static_assert((B_KB_BYTES % 1024) == 0, "swizzle atoms must stay 1024-B aligned");
 };
 
 struct Ctl {
@@ -144,9 +164,13 @@ __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, uint3
 
 // The whole BN-column accumulator row of this thread in one TMEM round trip.
 __device__ __forceinline__ void tmem_ld_tile(uint32_t taddr, float (&v)[128]) { tmem_ld128(taddr, v); }
+__device__ __forceinline__ void tmem_ld_tile(uint32_t taddr, float (&v)[96]) { tmem_ld96(taddr, v); }
 __device__ __forceinline__ void tmem_ld_tile(uint32_t taddr, float (&v)[64]) { tmem_ld64(taddr, v); }
+__device__ __forceinline__ void tmem_ld_tile(uint32_t taddr, float (&v)[48]) { tmem_ld48(taddr, v); }
+__device__ __forceinline__ void tmem_ld_tile(uint32_t taddr, float (&v)[32]) { tmem_ld32(taddr, v); }
 
 struct TcParams {
+  const uint16_t* a_ptr;   // A operand rows: q ([B][R][d]) in pass 1, k_ctx ([B][n_c][d]) in pass 2
   float* scores;
   float* lse2;
   uint32_t* status;
@@ -158,13 +182,13 @@ struct TcParams {
 
 template <int D, bool PASS2>
 __global__ void __launch_bounds__(kThreads, 1)
-    score_tc_kernel(const __grid_constant__ CUtensorMap amap,
-                    const __grid_constant__ CUtensorMap bmap0,
+    score_tc_kernel(const __grid_constant__ CUtensorMap bmap0,
                     const __grid_constant__ CUtensorMap bmap1, const TcParams p) {
   using Lay = TcLayout<D>;
   constexpr int BN = Lay::BN;
   constexpr int STAGES = Lay::STAGES;
   constexpr int KB = Lay::KB;
+  constexpr int CH = Lay::CH;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -199,16 +223,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   if (threadIdx.x == 0) {
-    mbar_init(a_full, 1);
+    mbar_init(a_full, nA * kBM);   // every thread of every active group stores its A row
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&b_full[s], 1);
-      mbar_init(&b_empty[s], 1);
+      mbar_init(&b_empty[s], nA);   // one commit per active MMA issuer
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], kBM);
     }
-    mbar_init(mma_done, 1);
+    mbar_init(mma_done, nA);
     // every thread of every active epilogue group releases each lse2 stage
     for (int s = 0; s < STAGES; ++s) mbar_init(&l_empty[s], nA * kBM);
     *abort_flag = 0;
@@ -227,17 +251,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ================================================================ TMA producer
     if (lane == 0) {
-      tma_prefetch_desc(&amap);
       tma_prefetch_desc(&bmap0);
       if (!PASS2) tma_prefetch_desc(&bmap1);
       const bool stall = p.test_stall != 0;
-      if (!stall) {
-        mbar_arrive_expect_tx(a_full, nA * Lay::A_BYTES);
-        for (int t = 0; t < nA; ++t)
-          for (int kb = 0; kb < KB; ++kb)
-            tma_load_3d(smem + Lay::OFF_A + t * Lay::A_BYTES + kb * Lay::A_KB_BYTES, &amap,
-                        a_full, kb * 64, a_row0 + t * kBM, b);
-      }
       int issued = 0;
 #pragma unroll 1
       for (int it = 0; !stall && it < n_b; ++it) {
@@ -261,46 +277,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         issued = it + 1;
       }
       // Drain: every copy this CTA started must land before shared memory is released.
-      if (!stall) wait_drain(a_full, 0, p.status);
       for (int s = 0; s < STAGES && s < issued; ++s) {
         const int last = s + ((issued - 1 - s) / STAGES) * STAGES;
         wait_drain(&b_full[s], (last / STAGES) & 1, p.status);
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ================================================================ MMA issuer
-    if (lane == 0) {
+  } else if (warp <= kATiles) {
+    // ================================================================ MMA issuers
+    const int t = warp - 1;                 // A tile (and epilogue group) of this issuer
+    if (lane == 0 && t < nA) {
       constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
-      const uint32_t a_base = smem_u32(smem + Lay::OFF_A);
       const uint32_t b_base = smem_u32(smem + Lay::OFF_B);
+      const uint32_t a_tmem = tmem_base + t * Lay::A_COLS;
       bool ok = wait_one(a_full, 0, ctl);
       tc_fence_after();
 #pragma unroll 1
       for (int it = 0; ok && it < n_b; ++it) {
         const int s = it % STAGES;
-        if (!wait_one(&b_full[s], (it / STAGES) & 1, ctl)) break;
-        tc_fence_after();
         const int buf = it & 1;
-        const uint32_t sph = (it >> 1) & 1;
-        for (int t = 0; t < nA; ++t) {
-          if (!wait_one(&s_empty[t * 2 + buf], sph ^ 1, ctl)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t d_tmem = tmem_base + (t * 2 + buf) * BN;
+        if (!wait_one(&b_full[s], (it / STAGES) & 1, ctl)) break;
+        if (!wait_one(&s_empty[t * 2 + buf], ((it >> 1) & 1) ^ 1, ctl)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + Lay::ACC0 + (t * 2 + buf) * BN;
 #pragma unroll
-          for (int kb = 0; kb < KB; ++kb) {
-            const uint64_t ad = sdesc_sw128(a_base + t * Lay::A_BYTES + kb * Lay::A_KB_BYTES);
-            const uint64_t bd = sdesc_sw128(b_base + s * Lay::B_BYTES + kb * Lay::B_KB_BYTES);
+        for (int kb = 0; kb < KB; ++kb) {
+          const uint64_t bd = sdesc_sw128(b_base + s * Lay::B_BYTES + kb * Lay::B_KB_BYTES);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_bf16_ss(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
-          }
-          umma_commit(&s_full[t * 2 + buf]);
+          for (int kk = 0; kk < 4; ++kk)   // K = 16 per MMA: 8 TMEM columns of A, 32 B of B
+            umma_bf16_ts(d_tmem, a_tmem + (kb * 4 + kk) * 8, bd + 2 * kk, idesc,
+                         (kb | kk) != 0);
         }
-        if (!ok) break;
+        umma_commit(&s_full[t * 2 + buf]);
         umma_commit(&b_empty[s]);
       }
       // Drain: all MMAs issued by this thread complete before TMEM is freed.
@@ -310,117 +318,177 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ================================================================ epilogue groups
-    const int t = (warp - 2) >> 2;          // A tile served by this group
+    // Group g = (A tile t, parity par): drains accumulator buffer (t, par), i.e.
+    // B tiles it = par, par + 2, ... of A tile t.  Four groups of four warps
+    // give each scheduler four epilogue warps to hide MUFU / TMEM latency.
+    const int g = (warp - 1 - kATiles) >> 2;
+    const int t = g >> 1, par = g & 1;
     const int quarter = warp & 3;           // TMEM lanes 32*quarter .. +31
     const int lrow = quarter * 32 + lane;   // row of the A tile
     const int arow = a_row0 + t * kBM + lrow;
     const float c = p.c;
+    float2* xchg = reinterpret_cast<float2*>(smem + Lay::OFF_XCHG) + t * kBM + lrow;
     if (t < nA) {
+      if (par == 0) {
+        // ---- this thread's A row into its TMEM lane (zeros past the operand's rows)
+        const uint4* src = reinterpret_cast<const uint4*>(
+            p.a_ptr + (static_cast<size_t>(b) * a_extent + arow) * D);
+        const bool in = arow < a_extent;
+        const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                t * Lay::A_COLS;
+#pragma unroll
+        for (int h = 0; h < D / 128; ++h) {   // 64 columns (128 bf16) per store
+          uint32_t w[64];
+#pragma unroll
+          for (int v4 = 0; v4 < 16; ++v4) {
+            const uint4 x = in ? __ldg(src + h * 16 + v4) : make_uint4(0, 0, 0, 0);
+            w[4 * v4 + 0] = x.x;
+            w[4 * v4 + 1] = x.y;
+            w[4 * v4 + 2] = x.z;
+            w[4 * v4 + 3] = x.w;
+          }
+          tmem_st64(a_lane + h * 64, w);
+        }
+        tc_fence_before();
+        mbar_arrive(a_full);
+      }
+      const uint32_t acc_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                Lay::ACC0 + (t * 2 + par) * BN;
       if (!PASS2) {
-        // ---------------- pass 1: online log-sum-exp over the row
+        // ---------------- pass 1: online log-sum-exp over the row (this parity's tiles)
         const int i_row = arow % p.n_in;
         float m = -INFINITY, l = 0.f;
 #pragma unroll 1
-        for (int it = 0; it < n_b; ++it) {
-          const int buf = it & 1;
-          if (!wait_warp(&s_full[t * 2 + buf], (it >> 1) & 1, ctl)) break;
+        for (int it = par; it < n_b; it += 2) {
+          if (!wait_warp(&s_full[t * 2 + par], (it >> 1) & 1, ctl)) break;
           tc_fence_after();
-          float v[BN];
-          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                 (t * 2 + buf) * BN;
-          tmem_ld_tile(taddr, v);
-          tc_fence_before();
-          mbar_arrive(&s_empty[t * 2 + buf]);
-          // masks: ragged context tail, causal self keys
-          if (it < n_kt_ctx) {
-            const int lim = p.n_c - it * BN;
-            if (lim < BN) {
-#pragma unroll
-              for (int j = 0; j < BN; ++j)
-                if (j >= lim) v[j] = -INFINITY;
+#pragma unroll 1
+          for (int ch = 0; ch < BN; ch += CH) {
+            float v[CH];
+            tmem_ld_tile(acc_lane + ch, v);
+            if (ch + CH == BN) {           // whole accumulator read: hand it back
+              tc_fence_before();
+              mbar_arrive(&s_empty[t * 2 + par]);
             }
-          } else {
-            const int lim = i_row - (it - n_kt_ctx) * BN;   // self key j' visible iff j' <= i
+            // masks: ragged context tail, causal self keys
+            if (it < n_kt_ctx) {
+              const int lim = p.n_c - it * BN - ch;
+              if (lim < CH) {
 #pragma unroll
-            for (int j = 0; j < BN; ++j)
-              if (j > lim) v[j] = -INFINITY;
-          }
-          float mx0 = v[0], mx1 = v[1];
-#pragma unroll
-          for (int j = 2; j + 3 < BN; j += 4) {
-            mx0 = fmax3(mx0, v[j], v[j + 1]);
-            mx1 = fmax3(mx1, v[j + 2], v[j + 3]);
-          }
-          mx0 = fmax3(mx0, mx1, fmaxf(v[BN - 2], v[BN - 1]));
-          const float m_new = fmaxf(m, mx0 * c);
-          const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-          // x = c*s - m in packed pairs; of every 8 pairs, kPolyPairs take 2^x on
-          // the FMA pipe and the rest on the MUFU unit, so both pipes share the work.
-          const float2 c2 = make_float2(c, c);
-          const float2 nm2 = make_float2(-m_use, -m_use);
-          float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int j = 0; j < BN; j += 16) {
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float2 x = ffma2(make_float2(v[j + 2 * q], v[j + 2 * q + 1]), c2, nm2);
-              float2 e;
-              if (q < kPolyPairs) {
-                e = exp2_poly2(x);
-              } else {
-                e.x = ex2_approx(x.x);
-                e.y = ex2_approx(x.y);
+                for (int j = 0; j < CH; ++j)
+                  if (j >= lim) v[j] = -INFINITY;
               }
-              if (q & 1)
-                acc1 = fadd2(acc1, e);
-              else
-                acc0 = fadd2(acc0, e);
+            } else {
+              const int lim = i_row - (it - n_kt_ctx) * BN - ch;   // visible iff j' <= i
+#pragma unroll
+              for (int j = 0; j < CH; ++j)
+                if (j > lim) v[j] = -INFINITY;
             }
+            // chunk maximum, 8 independent chains
+            float mx[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mx[k] = fmaxf(v[2 * k], v[2 * k + 1]);
+#pragma unroll
+            for (int j = 16; j < CH; j += 16) {
+#pragma unroll
+              for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], v[j + 2 * k], v[j + 2 * k + 1]);
+            }
+            const float mxa = fmax3(mx[0], mx[1], mx[2]), mxb = fmax3(mx[3], mx[4], mx[5]);
+            const float m_new = fmaxf(m, fmax3(mxa, mxb, fmaxf(mx[6], mx[7])) * c);
+            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+            // x = c*s - m in packed pairs; of every 8 pairs, kPolyPairs take 2^x on
+            // the FMA pipe and the rest on the MUFU unit.
+            const float2 c2 = make_float2(c, c);
+            const float2 nm2 = make_float2(-m_use, -m_use);
+            float2 acc[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int j = 0; j < CH; j += 16) {
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const float2 x = ffma2(make_float2(v[j + 2 * q], v[j + 2 * q + 1]), c2, nm2);
+                float2 e;
+                if (q < kPolyPairs) {
+                  e = exp2_poly2(x);
+                } else {
+                  e.x = ex2_approx(x.x);
+                  e.y = ex2_approx(x.y);
+                }
+                acc[q & 3] = fadd2(acc[q & 3], e);
+              }
+            }
+            const float2 s4 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+            l = fmaf(l, ex2_approx(m - m_use), s4.x + s4.y);
+            m = m_new;
           }
-          l = fmaf(l, ex2_approx(m - m_use), (acc0.x + acc0.y) + (acc1.x + acc1.y));
-          m = m_new;
         }
-        if (!*abort_flag && arow < p.R_pad)
-          p.lse2[static_cast<size_t>(b) * p.R_pad + arow] =
-              (arow < p.R) ? m + lg2_approx(l) : INFINITY;
+        // merge the two parities' (m, l) of this row; parity 0 writes lse2
+        if (par == 1) *xchg = make_float2(m, l);
+        named_barrier_sync(1 + t, 2 * kBM);
+        if (par == 0 && !*abort_flag && arow < p.R_pad) {
+          const float2 o = *xchg;
+          const float M = fmaxf(m, o.x);
+          float lse;
+          if (M == -INFINITY) {
+            lse = -INFINITY;
+          } else {
+            const float lt = l * ex2_approx(m - M) + o.y * ex2_approx(o.x - M);
+            lse = M + lg2_approx(lt);
+          }
+          p.lse2[static_cast<size_t>(b) * p.R_pad + arow] = (arow < p.R) ? lse : INFINITY;
+        }
       } else {
         // ---------------- pass 2: running max over query rows of c*s - lse2
         float best = -INFINITY;
 #pragma unroll 1
-        for (int it = 0; it < n_b; ++it) {
-          const int buf = it & 1;
+        for (int it = par; it < n_b; it += 2) {
           const int st = it % STAGES;
           // The stage's lse2 bytes landed with b_full; the stage cannot be refilled
           // before this group releases l_empty, so this phase is still the latest.
           if (!wait_warp(&b_full[st], (it / STAGES) & 1, ctl)) break;
-          if (!wait_warp(&s_full[t * 2 + buf], (it >> 1) & 1, ctl)) break;
+          if (!wait_warp(&s_full[t * 2 + par], (it >> 1) & 1, ctl)) break;
           tc_fence_after();
-          float v[BN];
-          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                 (t * 2 + buf) * BN;
-          tmem_ld_tile(taddr, v);
-          tc_fence_before();
-          mbar_arrive(&s_empty[t * 2 + buf]);
-          const float4* L4 = reinterpret_cast<const float4*>(smem + Lay::OFF_L + st * Lay::L_BYTES);
-          float b0 = best, b1 = -INFINITY;
+          const float4* L4 =
+              reinterpret_cast<const float4*>(smem + Lay::OFF_L + st * Lay::L_BYTES);
+#pragma unroll 1
+          for (int ch = 0; ch < BN; ch += CH) {
+            float v[CH];
+            tmem_ld_tile(acc_lane + ch, v);
+            if (ch + CH == BN) {
+              tc_fence_before();
+              mbar_arrive(&s_empty[t * 2 + par]);
+            }
+            float b0 = best, b1 = -INFINITY;
 #pragma unroll
-          for (int j = 0; j < BN; j += 4) {
-            const float4 L = L4[j / 4];   // same address in every lane: broadcast
-            b0 = fmax3(b0, fmaf(v[j + 0], c, -L.x), fmaf(v[j + 1], c, -L.y));
-            b1 = fmax3(b1, fmaf(v[j + 2], c, -L.z), fmaf(v[j + 3], c, -L.w));
+            for (int j = 0; j < CH; j += 4) {
+              const float4 L = L4[(ch + j) / 4];   // same address in every lane: broadcast
+              b0 = fmax3(b0, fmaf(v[j + 0], c, -L.x), fmaf(v[j + 1], c, -L.y));
+              b1 = fmax3(b1, fmaf(v[j + 2], c, -L.z), fmaf(v[j + 3], c, -L.w));
+            }
+            best = fmaxf(b0, b1);
           }
-          best = fmaxf(b0, b1);
           mbar_arrive(&l_empty[st]);
         }
-        if (!*abort_flag && arow < p.n_c) {
+        if (par == 1) xchg->x = best;
+        named_barrier_sync(1 + t, 2 * kBM);
+        if (par == 0 && !*abort_flag && arow < p.n_c) {
+          const float bb = fmaxf(best, xchg->x);
           float* dst = p.scores + static_cast<size_t>(b) * p.n_c + arow;
-          *dst = fmaxf(*dst, ex2_approx(best));
+          *dst = fmaxf(*dst, ex2_approx(bb));
         }
       }
-    } else if (!PASS2) {
+    } else if (!PASS2 && par == 0) {
       // A tile beyond the query rows: pad the log-sum-exp buffer with +inf so
       // that padded columns never win the pass-2 maximum.
       if (arow < p.R_pad) p.lse2[static_cast<size_t>(b) * p.R_pad + arow] = INFINITY;
+    }
+    if (!PASS2 && blockIdx.x == gridDim.x - 1) {
+      // Pass 2 reads whole BN-row tiles of lse2, up to the padded row count:
+      // rows past this grid's last tile are padding too.
+      for (int r = gridDim.x * kATiles * kBM + (threadIdx.x - 32 * (1 + kATiles)); r < p.R_pad;
+           r += kEpiThreads)
+        p.lse2[static_cast<size_t>(b) * p.R_pad + r] = INFINITY;
     }
   }
 
@@ -479,12 +547,13 @@ static cudaError_t launch_tc(const ScoreArgs& a, cudaStream_t s, int* launches) 
   e = cudaFuncSetAttribute(score_tc_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Lay::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
-  CUtensorMap qmap, kmap, smap;
-  if (!make_map(&qmap, a.q, a.B, a.R, D, kBM) ||  // A box for pass 1
-      !make_map(&kmap, a.k_ctx, a.B, a.n_c, D, Lay::BN) ||
+  // B operands only: A rows go straight from global memory into TMEM.
+  CUtensorMap kmap, smap;
+  if (!make_map(&kmap, a.k_ctx, a.B, a.n_c, D, Lay::BN) ||
       !make_map(&smap, a.k_self, a.B, a.n_in, D, Lay::BN))
     return cudaErrorInvalidValue;
   TcParams p;
+  p.a_ptr = static_cast<const uint16_t*>(a.q);
   p.scores = a.scores;
   p.lse2 = a.lse2;
   p.status = a.status;
@@ -499,20 +568,19 @@ static cudaError_t launch_tc(const ScoreArgs& a, cudaStream_t s, int* launches) 
 
   if (a.passes & 1) {
     dim3 g1((a.R + kATiles * kBM - 1) / (kATiles * kBM), a.B);
-    score_tc_kernel<D, false><<<g1, kThreads, Lay::SMEM_ALLOC, s>>>(qmap, kmap, smap, p);
+    score_tc_kernel<D, false><<<g1, kThreads, Lay::SMEM_ALLOC, s>>>(kmap, smap, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (launches) *launches += 1;
   }
   if (!(a.passes & 2)) return cudaSuccess;
 
-  // pass 2: A = context key tiles (box 128 rows), B = query row tiles (box BN rows)
-  CUtensorMap kmapA, qmapB;
-  if (!make_map(&kmapA, a.k_ctx, a.B, a.n_c, D, kBM) ||
-      !make_map(&qmapB, a.q, a.B, a.R, D, Lay::BN))
-    return cudaErrorInvalidValue;
+  // pass 2: A = context key tiles (TMEM), B = query row tiles (box BN rows)
+  CUtensorMap qmapB;
+  if (!make_map(&qmapB, a.q, a.B, a.R, D, Lay::BN)) return cudaErrorInvalidValue;
+  p.a_ptr = static_cast<const uint16_t*>(a.k_ctx);
   dim3 g2((a.n_c + kATiles * kBM - 1) / (kATiles * kBM), a.B);
-  score_tc_kernel<D, true><<<g2, kThreads, Lay::SMEM_ALLOC, s>>>(kmapA, qmapB, qmapB, p);
+  score_tc_kernel<D, true><<<g2, kThreads, Lay::SMEM_ALLOC, s>>>(qmapB, qmapB, p);
   e = cudaGetLastError();
   if (e == cudaSuccess && launches) *launches += 1;
   return e;

@@ -157,7 +157,7 @@ def read_lse(workspace: torch.Tensor, B: int, G: int, n_in: int) -> torch.Tensor
     """Natural-log row normalisers the last pass-1 launch left in the workspace,
     [B][G*n_in] (a view into the workspace's padded buffer, converted)."""
     R = G * n_in
-    R_pad = (R + 255) // 256 * 256
+    R_pad = (R + 767) // 768 * 768
     lse2 = workspace[256:256 + B * R_pad * 4].view(torch.float32).view(B, R_pad)[:, :R]
     return lse2 * 0.6931471805599453
 

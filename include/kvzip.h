@@ -57,7 +57,7 @@ typedef enum {
 /* ------------------------------------------------------------------ scoring */
 
 /* Bytes of workspace kvzip_score_chunk needs for B units of G*n_in query rows:
- * a 256-byte status header plus one float per query row, rows padded to 256. */
+ * a 256-byte status header plus one float per query row, rows padded to 768. */
 size_t kvzip_score_workspace_size(int B, int G, int n_in);
 
 /*

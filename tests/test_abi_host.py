@@ -64,7 +64,7 @@ def test_keep_count_rejects(kz):
 
 
 def test_workspace_sizes(kz):
-    assert kz.score_workspace_size(256, 4, 2064) == 256 + 256 * (math.ceil(8256 / 256) * 256) * 4
+    assert kz.score_workspace_size(256, 4, 2064) == 256 + 256 * (math.ceil(8256 / 768) * 768) * 4
     assert kz.select_workspace_size(33554432, 256) > 0
     assert kz.compact_workspace_size(256, 131072) > 0
 
