@@ -18,4 +18,5 @@ from .kvzip_oracle import (  # noqa: F401
     select,
     compact,
     head_scores,
+    decode_attention,
 )

@@ -41,6 +41,9 @@ design notes):
 7. k = ceil(r * N) computed in IEEE double; among equal scores the lower flat
    index f = (l * H + h) * n_c + j is kept first.
 8. Compacted caches are packed head-major, positions ascending in each head.
+9. Decoding over a compressed cache attends each query head to its KV head's
+   kept rows only (standard softmax attention, scale 1/sqrt(d)); a head with
+   no kept rows returns zeros.
 
 Everything is float64 on inputs converted exactly from their storage type
 (bf16 and fp32 values are exactly representable in float64).
@@ -202,3 +205,29 @@ def head_scores(S, L: int, H: int) -> np.ndarray:
     """Head-level score max_j S[l, h, j] (rebuttal, answer on how head-level
     scores for the DuoAttention comparison were computed)."""
     return _f64(S).reshape(L, H, -1).max(axis=2)
+
+
+def decode_attention(q, k_packed, v_packed, offsets, scale: float | None = None):
+    """One decoding step of attention over the compressed, per-head variable-length
+    cache (rebuttal, computational-efficiency table: decoding attention over the
+    cache kept at each ratio).
+
+    q: [n_heads, G, d] (the G query heads of each KV head); k_packed, v_packed:
+    [total, d] packed head-major; offsets: [n_heads+1].
+    Returns o [n_heads, G, d] float64: o[h, g] = softmax(scale * K_h q_g) @ V_h over
+    head h's kept rows (reading 9: zeros for an empty head).
+    """
+    q = _f64(q)
+    K = _f64(k_packed)
+    V = _f64(v_packed)
+    n_heads, G, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = np.zeros((n_heads, G, d))
+    for h in range(n_heads):
+        a, b = int(offsets[h]), int(offsets[h + 1])
+        if b == a:
+            continue
+        logits = scale * (q[h] @ K[a:b].T)                 # [G, n_h]
+        out[h] = softmax_rows(logits) @ V[a:b]
+    return out

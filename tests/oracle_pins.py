@@ -307,8 +307,60 @@ def pin_kv_size_table(o):
         assert round(32.7 * nbytes / full, 1) == gb, (ratio, 32.7 * nbytes / full, gb)
 
 
+# --------------------------------------------------------- decode attention pins
+
+def pin_decode_closed_forms(o):
+    """Decode attention: a head with one kept row returns that row's V; zero
+    queries average the head's V rows; an empty head returns zeros; a
+    dominant aligned key returns its V row."""
+    r = _rng(60)
+    d, G = 8, 3
+    K = r.standard_normal((7, d))
+    V = r.standard_normal((7, d))
+    offsets = np.array([0, 1, 1, 4, 7])          # heads of 1, 0, 3, 3 rows
+    q = r.standard_normal((4, G, d))
+    out = o.decode_attention(q, K, V, offsets)
+    assert np.allclose(out[0], V[0], rtol=0, atol=1e-14)
+    assert np.all(out[1] == 0)
+    out0 = o.decode_attention(np.zeros((4, G, d)), K, V, offsets)
+    assert np.allclose(out0[2], V[1:4].mean(axis=0), rtol=0, atol=1e-14)
+    assert np.allclose(out0[3], V[4:7].mean(axis=0), rtol=0, atol=1e-14)
+    K2 = K.copy()
+    K2[5] = 200.0 * q[3, 1] / np.linalg.norm(q[3, 1])
+    out2 = o.decode_attention(q, K2, V, offsets)
+    assert np.allclose(out2[3, 1], V[5], rtol=0, atol=1e-9)
+
+
+def pin_decode_matches_dense_over_kept(o):
+    """Decode attention over the compacted cache equals dense attention over
+    the full cache with evicted keys masked out (pure-Python loops)."""
+    r = _rng(61)
+    n_heads, n_c, d, G = 3, 9, 4, 2
+    K = r.standard_normal((n_heads, n_c, d))
+    V = r.standard_normal((n_heads, n_c, d))
+    s = r.random(n_heads * n_c).astype(np.float32)
+    kk = o.keep_count(0.5, s.size)
+    keep, offsets, _ = o.select(s, kk, n_heads)
+    ko, vo, _ = o.compact(K, V, keep, offsets)
+    q = r.standard_normal((n_heads, G, d))
+    got = o.decode_attention(q, ko, vo, offsets)
+    keep = keep.reshape(n_heads, n_c)
+    for h in range(n_heads):
+        for g in range(G):
+            ls = [(sum(float(a) * float(b) for a, b in zip(q[h, g], K[h, j])) / math.sqrt(d), j)
+                  for j in range(n_c) if keep[h, j]]
+            if not ls:
+                assert np.all(got[h, g] == 0)
+                continue
+            mx = max(x for x, _ in ls)
+            z = sum(math.exp(x - mx) for x, _ in ls)
+            want = [sum(math.exp(x - mx) / z * float(V[h, j, t]) for x, j in ls) for t in range(d)]
+            assert np.allclose(got[h, g], want, rtol=1e-12, atol=1e-14)
+
+
 SCORING_PINS = [pin_row_sums_and_range, pin_uniform_queries, pin_logistic, pin_dominant_key,
                 pin_bruteforce_unchunked, pin_invariants, pin_rows_see_own_prefix]
 SELECT_PINS = [pin_keep_count, pin_select_properties, pin_select_bruteforce]
 COMPACT_PINS = [pin_compact, pin_kv_size_table]
-ALL_PINS = SCORING_PINS + SELECT_PINS + COMPACT_PINS
+DECODE_PINS = [pin_decode_closed_forms, pin_decode_matches_dense_over_kept]
+ALL_PINS = SCORING_PINS + SELECT_PINS + COMPACT_PINS + DECODE_PINS

@@ -142,10 +142,24 @@ def _mut_positions_descending(m):
     m.compact = compact
 
 
+def _mut_decode_no_scale(m):
+    orig = m.decode_attention
+    m.decode_attention = lambda q, k, v, off, scale=None: orig(q, k, v, off, 1.0)
+
+
+def _mut_decode_wrong_head(m):
+    orig = m.decode_attention
+
+    def dec(q, k, v, off, scale=None):
+        q = np.asarray(q)
+        return orig(q[::-1].copy(), k, v, off, scale)[::-1].copy()
+    m.decode_attention = dec
+
+
 MUTANTS = [_mut_drop_diagonal, _mut_anticausal, _mut_row_order, _mut_no_self_in_normaliser,
            _mut_no_scale, _mut_mean, _mut_sum_over_chunks, _mut_transposed_keys,
            _mut_floor_count, _mut_tie_high_index, _mut_uniform_head_budget,
-           _mut_positions_descending]
+           _mut_positions_descending, _mut_decode_no_scale, _mut_decode_wrong_head]
 
 
 @pytest.mark.parametrize("mutate", MUTANTS, ids=lambda f: f.__name__)
