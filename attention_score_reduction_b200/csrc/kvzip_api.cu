@@ -232,4 +232,41 @@ kvzip_status kvzip_head_scores(const float* scores, int64_t n_heads, int64_t n_c
   return from_cuda(e);
 }
 
+size_t kvzip_decode_workspace_size(int64_t n_heads, int G, int d) {
+  if (n_heads <= 0 || G <= 0 || d <= 0) return 0;
+  return kvzip::decode_ws_bytes(n_heads, G, d);
+}
+
+kvzip_status kvzip_decode_attention(const void* q, const void* k_packed, const void* v_packed,
+                                    const int64_t* offsets, int64_t n_heads, int G, int d,
+                                    float scale, float* out, void* workspace, size_t ws_bytes,
+                                    void* stream) {
+  if (n_heads <= 0 || n_heads > 65535 || G <= 0) return KVZIP_ERR_INVALID_ARG;
+  if (d != 128 && d != 256) return d > 0 ? KVZIP_ERR_UNSUPPORTED : KVZIP_ERR_INVALID_ARG;
+  if (G != 1 && G != 2 && G != 4 && G != 5 && G != 8) return KVZIP_ERR_UNSUPPORTED;
+  if (!q || !offsets || !out || !workspace) return KVZIP_ERR_INVALID_ARG;
+  if ((k_packed == nullptr) != (v_packed == nullptr)) return KVZIP_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_packed, 16) || !aligned(v_packed, 16) ||
+      !aligned(offsets, 8) || !aligned(out, 4) || !aligned(workspace, 256))
+    return KVZIP_ERR_INVALID_ARG;
+  if (ws_bytes < kvzip_decode_workspace_size(n_heads, G, d)) return KVZIP_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || std::isinf(scale)) scale = 1.0f / std::sqrt(static_cast<float>(d));
+  kvzip::DecodeArgs a;
+  a.q = q;
+  a.k = k_packed;
+  a.v = v_packed;
+  a.offsets = offsets;
+  a.n_heads = n_heads;
+  a.G = G;
+  a.d = d;
+  a.scale = scale;
+  a.out = out;
+  a.ws = workspace;
+  a.timeout_ns = g_timeout_ns.load();
+  int launches = 0;
+  cudaError_t e = kvzip::launch_decode(a, static_cast<cudaStream_t>(stream), &launches);
+  if (e == cudaSuccess) g_last_launches.store(launches);
+  return from_cuda(e);
+}
+
 }  // extern "C"

@@ -70,4 +70,22 @@ cudaError_t launch_compact(const CompactArgs& a, cudaStream_t s, int* launches);
 cudaError_t launch_head_scores(const float* scores, int64_t n_heads, int64_t n_c, float* out,
                                cudaStream_t s, int* launches);
 
+struct DecodeArgs {
+  const void* q;          // [n_heads][G][d] bf16
+  const void* k;          // [total][d] bf16, packed head-major
+  const void* v;
+  const int64_t* offsets; // [n_heads + 1]
+  int64_t n_heads;
+  int G, d;
+  float scale;
+  float* out;             // [n_heads][G][d] fp32
+  void* ws;               // 256-byte status header, then the split partials
+  uint64_t timeout_ns;
+};
+constexpr size_t kDecodeWsHeader = 256;
+int decode_splits(int64_t n_heads);
+size_t decode_ml_bytes(int64_t n_heads, int G);
+size_t decode_ws_bytes(int64_t n_heads, int G, int d);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, int* launches);
+
 }  // namespace kvzip

@@ -378,6 +378,12 @@ __device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
   return f2_unpack(r);
 }
 
+__device__ __forceinline__ int imad_lo(int a, int b, int c) {  // a * b + c (mod 2^32)
+  int r;
+  asm("mad.lo.s32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+
 // 2^x on the FMA pipe for x <= 0 (x below -125 is clamped; 2^-125 is negligible
 // next to the row maximum's 2^0).  Cody-Waite style split x = n + f with n the
 // nearest integer (added into the exponent field) and f in [-1/2, 1/2]; 2^f by
@@ -395,8 +401,9 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                    make_float2(0.2426113784313202f, 0.2426113784313202f));
   p = ffma2(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
   p = ffma2(p, f, make_float2(0.9999279975891113f, 0.9999279975891113f));
-  p.x = __int_as_float(__float_as_int(p.x) + (__float_as_int(j.x) << 23));
-  p.y = __int_as_float(__float_as_int(p.y) + (__float_as_int(j.y) << 23));
+  // p * 2^n: add n (the low bits of j) into the exponent field, one IMAD each
+  p.x = __int_as_float(imad_lo(__float_as_int(j.x), 1 << 23, __float_as_int(p.x)));
+  p.y = __int_as_float(imad_lo(__float_as_int(j.y), 1 << 23, __float_as_int(p.y)));
   return p;
 }
 

@@ -47,6 +47,8 @@ def _load() -> ctypes.CDLL:
         "kvzip_compact_workspace_size": (sz, [i64, i32]),
         "kvzip_compact": (i32, [vp, vp, vp, vp, i64, i32, i32, vp, vp, vp, vp, sz, vp]),
         "kvzip_head_scores": (i32, [vp, i64, i64, vp, vp]),
+        "kvzip_decode_workspace_size": (sz, [i64, i32, i32]),
+        "kvzip_decode_attention": (i32, [vp, vp, vp, vp, i64, i32, i32, f32, vp, vp, sz, vp]),
         "kvzip_last_launch_count": (i32, []),
         "kvzip_status_string": (ctypes.c_char_p, [i32]),
     }
@@ -238,6 +240,36 @@ def head_scores(scores: torch.Tensor, out: torch.Tensor | None = None, stream=No
     out = torch.empty(n_heads, dtype=torch.float32, device=scores.device) if out is None else out
     _check(_lib.kvzip_head_scores(_ptr(scores), n_heads, n_c, _ptr(out), _stream(stream)),
            "kvzip_head_scores")
+    return out
+
+
+# ---------------------------------------------------------------- decode attention
+
+def decode_workspace_size(n_heads: int, G: int, d: int) -> int:
+    return int(_lib.kvzip_decode_workspace_size(n_heads, G, d))
+
+
+def decode_attention(q: torch.Tensor, k_packed: torch.Tensor, v_packed: torch.Tensor,
+                     offsets: torch.Tensor, out: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None, scale: float = 0.0, stream=None):
+    """softmax(scale * K_h q) V_h per KV head over its kept rows.
+
+    q [n_heads][G][d] bf16; k_packed / v_packed [total][d] bf16; offsets int64
+    [n_heads+1].  Returns out [n_heads][G][d] float32.
+    """
+    _dev_contig("q", q, torch.bfloat16)
+    n_heads, G, d = q.shape
+    dev = q.device
+    out = torch.empty(n_heads, G, d, dtype=torch.float32, device=dev) if out is None else out
+    if workspace is None:
+        workspace = torch.zeros(max(decode_workspace_size(n_heads, G, d), 256), dtype=torch.uint8,
+                                device=dev)
+    kp = k_packed if k_packed.numel() else None
+    vp = v_packed if v_packed.numel() else None
+    _check(_lib.kvzip_decode_attention(_ptr(q), _ptr(kp), _ptr(vp), _ptr(offsets), n_heads, G, d,
+                                       float(scale), _ptr(out), _ptr(workspace),
+                                       workspace.numel(), _stream(stream)),
+           "kvzip_decode_attention")
     return out
 
 

@@ -128,16 +128,17 @@ def _keys(wl: Workload, units: int, n: int, g: torch.Generator, device,
         row = row * torch.exp(wl.lognormal_sigma * z)
     if with_sinks and wl.sinks > 0:
         row[:, : min(wl.sinks, n)] = row[:, : min(wl.sinks, n)] * wl.sink_scale
-    return k * row
+    return k.mul_(row)   # in place: the full-size float32 keys are tens of GB
 
 
 def context_kv(wl: Workload, device="cpu", units: int | None = None):
     """(k_ctx, v): ``[units][n_c][d]`` each; k in the workload dtype, v in bf16."""
     u = wl.units if units is None else units
     k = _keys(wl, u, wl.n_c, _gen(device, _seed(wl, _T_KCTX)), device, with_sinks=True)
+    k = k.to(_storage(wl, "k"))
     v = torch.randn(u, wl.n_c, wl.d, generator=_gen(device, _seed(wl, _T_V)),
                     device=device, dtype=torch.float32)
-    return k.to(_storage(wl, "k")), v.to(torch.bfloat16)
+    return k, v.to(torch.bfloat16)
 
 
 def context_keys(wl: Workload, device="cpu", units: int | None = None) -> torch.Tensor:

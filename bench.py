@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode-attention table")
     return ap.parse_args()
 
 
@@ -285,6 +286,11 @@ def main():
         "step_pct_bf16_tc_peak": 100.0 * executed_tf / peak_tf,
     }
 
+    # ------------------------------------------------------------ decode over the kept cache
+    decode = None
+    if not args.no_decode:
+        decode = run_decode(wl, comp, k_ctx, v, dev, peaks)
+
     # ------------------------------------------------------------ end to end
     e2e = None
     if not args.no_e2e:
@@ -296,7 +302,8 @@ def main():
            "data": "synthetic", "config": config_dict(wl, r), "parallelism":
            f"{world} independent contexts, one per GPU", "clocks": clocks,
            "gpu_launches": launches, "roofline": roofline, "kernels": kernels,
-           "pct_bf16_tc_peak": kernels["step_pct_bf16_tc_peak"], "e2e": e2e}
+           "pct_bf16_tc_peak": kernels["step_pct_bf16_tc_peak"], "e2e": e2e,
+           "decode_attention": decode}
 
     # free device memory before the CPU baseline allocates host buffers
     del chunks, k_ctx, v, comp
@@ -312,6 +319,51 @@ def main():
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+def run_decode(wl, comp, k_ctx, v, dev, peaks, ratios=(1.0, 0.8, 0.6, 0.4, 0.2), iters=20):
+    """Decode-attention latency over layer 0's cache kept at each ratio.
+
+    The analogue of the rebuttal's decoding-efficiency table (latency and cache
+    size against the kept ratio): layer 0's H heads are ranked by the scores of
+    the last step, compacted at ratio r, and one decoding step of attention
+    (G query heads per KV head) reads the kept rows.  L2 is flushed (a 256 MB
+    write) before every timed launch.
+    """
+    from attention_score_reduction_b200 import kvzip as kz
+    H, n_c, d, G = wl.H, wl.n_c, wl.d, wl.G
+    s0 = comp.scores[:H].contiguous().view(-1)
+    k0, v0 = k_ctx[:H].contiguous(), v[:H].contiguous()
+    g = torch.Generator(device=dev)
+    g.manual_seed(synth.BASE_SEED + 5)
+    q = torch.randn(H, G, d, generator=g, device=dev).to(torch.bfloat16)
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
+    ws = torch.zeros(kz.decode_workspace_size(H, G, d), dtype=torch.uint8, device=dev)
+    out = torch.empty(H, G, d, dtype=torch.float32, device=dev)
+    rows = []
+    for r in ratios:
+        kept = kz.keep_count(r, s0.numel())
+        keep, off, _ = kz.select(s0, kept, H)
+        ko, vo, _ = kz.compact(k0, v0, keep, off, kept, want_pos=False)
+        ms = 0.0
+        for i in range(iters + 3):
+            flush.fill_(i & 0xff)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            kz.decode_attention(q, ko, vo, off, out, ws)
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                ms += e0.elapsed_time(e1)
+        ms /= iters
+        nbytes = kept * d * 2 * 2 + q.numel() * 2 + out.numel() * 4
+        rows.append((r, ms, kept * d * 2 * 2, nbytes / (ms * 1e-3) / 1e9))
+    full = rows[0][1]
+    return {"workload": f"layer 0: {H} KV heads x G={G}, d={d}, {n_c} positions, one decoding step",
+            "r": [x[0] for x in rows], "ms": [x[1] for x in rows],
+            "kv_bytes": [x[2] for x in rows], "gbs": [x[3] for x in rows],
+            "frac_of_hbm": [x[3] / peaks["hbm_gbs"] for x in rows],
+            "speedup_vs_full": [full / x[1] for x in rows], "l2": "flushed before each launch"}
 
 
 def _pinned_like(t):

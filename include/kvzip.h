@@ -201,6 +201,32 @@ kvzip_status kvzip_compact(const void* k, const void* v, const uint8_t* keep,
                            void* k_out, void* v_out, int32_t* pos_out, void* workspace,
                            size_t ws_bytes, void* stream);
 
+/* -------------------------------------------------------- decode attention */
+
+/* Bytes of workspace kvzip_decode_attention needs.  Like the scoring
+ * workspace it starts with a sticky status word (zero it before first use;
+ * kvzip_workspace_status reads and clears it). */
+size_t kvzip_decode_workspace_size(int64_t n_heads, int G, int d);
+
+/*
+ * One decoding step of attention over the compressed cache from kvzip_compact
+ * (rebuttal, decoding-efficiency table: decoding attention latency falls with
+ * the kept ratio because only kept KV pairs are read).  For every KV head h
+ * and each of its G query heads g:
+ *   out[h][g] = softmax(scale * K_h q[h][g]) V_h
+ * over head h's kept rows K_h = k_packed[offsets[h] : offsets[h+1]] (same for V).
+ * A head with no kept rows gives zeros.
+ *   q         [n_heads][G][d] bf16, 16-byte aligned.
+ *   k_packed, v_packed  [offsets[n_heads]][d] bf16 (may be NULL only if nothing is kept).
+ *   offsets   [n_heads + 1] int64 (device).
+ *   G         1, 2, 4, 5 or 8; d 128 or 256; scale <= 0 selects 1/sqrt(d).
+ *   out       [n_heads][G][d] float32.
+ */
+kvzip_status kvzip_decode_attention(const void* q, const void* k_packed, const void* v_packed,
+                                    const int64_t* offsets, int64_t n_heads, int G, int d,
+                                    float scale, float* out, void* workspace, size_t ws_bytes,
+                                    void* stream);
+
 /* ------------------------------------------------------------ head scores */
 
 /*
