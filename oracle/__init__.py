@@ -19,4 +19,9 @@ from .kvzip_oracle import (  # noqa: F401
     compact,
     head_scores,
     decode_attention,
+    unit_chunk_colsums,
+    score_chunk_sum,
+    token_scores,
+    select_per_head,
+    expand_keep,
 )

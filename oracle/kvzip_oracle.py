@@ -44,6 +44,11 @@ design notes):
 9. Decoding over a compressed cache attends each query head to its KV head's
    kept rows only (standard softmax attention, scale 1/sqrt(d)); a head with
    no kept rows returns zeros.
+10. Sum aggregation (the rebuttal's average-aggregation ablation; sum and
+    average rank pairs identically) adds each chunk's column sums of the same
+    softmax instead of taking maxima.
+11. Uniform head budgets give every head the same k_h = ceil(r * n_c) pairs,
+    ranked inside the head with the same tie rule.
 
 Everything is float64 on inputs converted exactly from their storage type
 (bf16 and fp32 values are exactly representable in float64).
@@ -231,3 +236,50 @@ def decode_attention(q, k_packed, v_packed, offsets, scale: float | None = None)
         logits = scale * (q[h] @ K[a:b].T)                 # [G, n_h]
         out[h] = softmax_rows(logits) @ V[a:b]
     return out
+
+
+def unit_chunk_colsums(q, k_ctx, k_self, scale: float | None = None):
+    """Sum aggregation for one unit and chunk: sum over rows of softmax[row, j], j < n_c
+    (rebuttal, answer on sum/average aggregation; reading 10)."""
+    k_ctx = _f64(k_ctx)
+    n_c, d = k_ctx.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    p = softmax_rows(chunk_logits(q, k_ctx, k_self, scale))
+    return p[:, :n_c].sum(axis=0)
+
+
+def score_chunk_sum(q, k_ctx, k_self, scores, scale: float | None = None):
+    """Sum-aggregation counterpart of score_chunk: scores += chunk column sums."""
+    for b in range(len(q)):
+        scores[b] += unit_chunk_colsums(q[b], k_ctx[b], k_self[b], scale)
+    return scores
+
+
+def token_scores(S):
+    """Token-level importance S[j] = max over (layer, head) of S[l, h, j]
+    (blog post section 4.3.3): one score per position, shared by all heads."""
+    return _f64(S).reshape(-1, np.asarray(S).shape[-1]).max(axis=0)
+
+
+def select_per_head(scores, k_h: int, n_heads: int):
+    """Uniform head budgets (reading 11): the k_h highest scores inside every
+    head, lower position first among equal scores.  Returns (keep, offsets)."""
+    s = np.asarray(scores).reshape(n_heads, -1)
+    n_c = s.shape[1]
+    if not (0 <= k_h <= n_c):
+        raise ValueError("k_h must lie in [0, n_c]")
+    keep = np.zeros_like(s, dtype=np.uint8)
+    for h in range(n_heads):
+        order = np.lexsort((np.arange(n_c), -s[h].astype(np.float64)))
+        keep[h, order[:k_h]] = 1
+    offsets = np.arange(n_heads + 1, dtype=np.int64) * k_h
+    return keep.reshape(-1), offsets
+
+
+def expand_keep(keep_pos, n_heads: int):
+    """A position mask shared by all heads, as a per-head mask and offsets."""
+    kp = np.asarray(keep_pos).astype(np.uint8).reshape(-1)
+    keep = np.tile(kp, n_heads)
+    offsets = np.arange(n_heads + 1, dtype=np.int64) * int(kp.sum())
+    return keep, offsets

@@ -358,9 +358,56 @@ def pin_decode_matches_dense_over_kept(o):
             assert np.allclose(got[h, g], want, rtol=1e-12, atol=1e-14)
 
 
+# ------------------------------------------------------------- variant pins
+
+def pin_sum_aggregation(o):
+    """Sum aggregation: Q = 0 gives S[j] = G * sum_i 1/(n_c + i + 1) (each row
+    is uniform over its n_c + i + 1 keys); column sums plus the self-key mass
+    account for every row's probability 1 (pure-Python check on a tiny case)."""
+    G, n_in, n_c, d = 3, 7, 11, 4
+    r = _rng(70)
+    k = r.standard_normal((1, n_c, d))
+    ks = r.standard_normal((1, n_in, d))
+    S = np.zeros((1, n_c))
+    o.score_chunk_sum(np.zeros((1, G, n_in, d)), k, ks, S)
+    want = G * sum(1.0 / (n_c + i + 1) for i in range(n_in))
+    assert np.allclose(S, want, rtol=1e-13, atol=0)
+    q = r.standard_normal((G, n_in, d))
+    cs = o.unit_chunk_colsums(q, k[0], ks[0])
+    self_mass = 0.0
+    for g in range(G):
+        for i in range(n_in):
+            lg = [float(q[g, i] @ k[0, j]) / 2.0 for j in range(n_c)] + \
+                 [float(q[g, i] @ ks[0, jp]) / 2.0 for jp in range(i + 1)]
+            mx = max(lg)
+            z = sum(math.exp(x - mx) for x in lg)
+            self_mass += sum(math.exp(x - mx) for x in lg[n_c:]) / z
+    assert abs(cs.sum() + self_mass - G * n_in) < 1e-12
+
+
+def pin_token_and_uniform_budgets(o):
+    """Token-level scores are the per-position max over heads; uniform budgets
+    keep exactly k_h per head, each head's kept set being its own top k_h
+    (checked by the defining property), and an all-heads position mask
+    expands to identical per-head masks."""
+    r = _rng(71)
+    S = (np.floor(r.random((4, 30)) * 6) / 6).astype(np.float32)
+    tok = o.token_scores(S)
+    assert np.array_equal(tok, S.max(axis=0).astype(np.float64))
+    keep, off = o.select_per_head(S.reshape(-1), 9, 4)
+    assert np.array_equal(off, [0, 9, 18, 27, 36])
+    for h in range(4):
+        _check_selection(S[h], 9, 1, keep.reshape(4, 30)[h], np.array([0, 9]), S[h][keep.reshape(4, 30)[h] == 1].min())
+    kp = np.zeros(30, np.uint8)
+    kp[[1, 5, 7]] = 1
+    ke, offe = o.expand_keep(kp, 4)
+    assert np.array_equal(ke.reshape(4, 30), np.tile(kp, (4, 1))) and offe[-1] == 12
+
+
 SCORING_PINS = [pin_row_sums_and_range, pin_uniform_queries, pin_logistic, pin_dominant_key,
                 pin_bruteforce_unchunked, pin_invariants, pin_rows_see_own_prefix]
 SELECT_PINS = [pin_keep_count, pin_select_properties, pin_select_bruteforce]
 COMPACT_PINS = [pin_compact, pin_kv_size_table]
 DECODE_PINS = [pin_decode_closed_forms, pin_decode_matches_dense_over_kept]
-ALL_PINS = SCORING_PINS + SELECT_PINS + COMPACT_PINS + DECODE_PINS
+VARIANT_PINS = [pin_sum_aggregation, pin_token_and_uniform_budgets]
+ALL_PINS = SCORING_PINS + SELECT_PINS + COMPACT_PINS + DECODE_PINS + VARIANT_PINS

@@ -156,10 +156,33 @@ def _mut_decode_wrong_head(m):
     m.decode_attention = dec
 
 
+def _mut_sum_without_self(m):
+    def colsums(q, k_ctx, k_self, scale=None):
+        k_ctx = np.asarray(k_ctx, np.float64)
+        if scale is None:
+            scale = 1 / math.sqrt(k_ctx.shape[1])
+        a = m.chunk_logits(q, k_ctx, k_self, scale)[:, :k_ctx.shape[0]]
+        return m.softmax_rows(a).sum(axis=0)
+    m.unit_chunk_colsums = colsums
+
+
+def _mut_per_head_tie_high(m):
+    def sph(scores, k_h, n_heads):
+        s = np.asarray(scores).reshape(n_heads, -1)
+        n_c = s.shape[1]
+        keep = np.zeros_like(s, dtype=np.uint8)
+        for h in range(n_heads):
+            order = np.lexsort((-np.arange(n_c), -s[h].astype(np.float64)))
+            keep[h, order[:k_h]] = 1
+        return keep.reshape(-1), np.arange(n_heads + 1, dtype=np.int64) * k_h
+    m.select_per_head = sph
+
+
 MUTANTS = [_mut_drop_diagonal, _mut_anticausal, _mut_row_order, _mut_no_self_in_normaliser,
            _mut_no_scale, _mut_mean, _mut_sum_over_chunks, _mut_transposed_keys,
            _mut_floor_count, _mut_tie_high_index, _mut_uniform_head_budget,
-           _mut_positions_descending, _mut_decode_no_scale, _mut_decode_wrong_head]
+           _mut_positions_descending, _mut_decode_no_scale, _mut_decode_wrong_head,
+           _mut_sum_without_self, _mut_per_head_tie_high]
 
 
 @pytest.mark.parametrize("mutate", MUTANTS, ids=lambda f: f.__name__)
