@@ -8,6 +8,7 @@
 // into an output zeroed first (0.0f is a lower bound of every score).
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 
 #include "kvzip_internal.h"
@@ -41,7 +42,49 @@ __global__ void __launch_bounds__(kHeadThreads)
   }
 }
 
+// Token-level scores: tok[j] = max over heads of scores[h][j] (blog post
+// section 4.3.3, a position kept or evicted in every head at once).
+__global__ void __launch_bounds__(256)
+    token_max_kernel(const float* __restrict__ s, int64_t n_heads, int64_t n_c, float* tok) {
+  for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < n_c;
+       j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float m = s[j];
+    for (int64_t h = 1; h < n_heads; ++h) m = fmaxf(m, s[h * n_c + j]);
+    tok[j] = m;
+  }
+}
+
+// keep[h][j] = keep_pos[j] for every head; offsets[h] = h * (kept positions).
+__global__ void __launch_bounds__(256)
+    expand_keep_kernel(const uint8_t* __restrict__ keep_pos, const int64_t* __restrict__ pos_off,
+                       int64_t n_heads, int64_t n_c, uint8_t* keep, int64_t* offsets) {
+  const int64_t total = n_heads * n_c;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (int64_t i = i0; i < total; i += stride) keep[i] = keep_pos[i % n_c] ? 1 : 0;
+  const int64_t kept = pos_off[1] - pos_off[0];
+  for (int64_t h = i0; h <= n_heads; h += stride) offsets[h] = h * kept;
+}
+
 }  // namespace
+
+cudaError_t launch_token_scores(const float* scores, int64_t n_heads, int64_t n_c, float* tok,
+                                cudaStream_t s, int* launches) {
+  const int64_t blocks = std::min<int64_t>((n_c + 255) / 256, 148 * 8);
+  token_max_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(scores, n_heads, n_c, tok);
+  if (launches) *launches += 1;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_expand_keep(const uint8_t* keep_pos, const int64_t* pos_off, int64_t n_heads,
+                               int64_t n_c, uint8_t* keep, int64_t* offsets, cudaStream_t s,
+                               int* launches) {
+  const int64_t blocks = std::min<int64_t>((n_heads * n_c + 255) / 256, 148 * 8);
+  expand_keep_kernel<<<static_cast<unsigned>(std::max<int64_t>(blocks, 1)), 256, 0, s>>>(
+      keep_pos, pos_off, n_heads, n_c, keep, offsets);
+  if (launches) *launches += 1;
+  return cudaGetLastError();
+}
 
 cudaError_t launch_head_scores(const float* scores, int64_t n_heads, int64_t n_c, float* out,
                                cudaStream_t s, int* launches) {

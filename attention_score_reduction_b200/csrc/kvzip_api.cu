@@ -53,7 +53,7 @@ size_t kvzip_score_workspace_size(int B, int G, int n_in) {
   return kvzip::kScoreWsHeader + static_cast<size_t>(B) * static_cast<size_t>(row_pad(R)) * 4;
 }
 
-static kvzip_status score_passes(int passes, kvzip_dtype dt, const void* q, const void* k_ctx,
+static kvzip_status score_passes(int passes, int sum_agg, kvzip_dtype dt, const void* q, const void* k_ctx,
                                  const void* k_self, float* scores, int B, int G, int n_in,
                                  int n_c, int d, float scale, void* workspace, size_t ws_bytes,
                                  void* stream) {
@@ -87,6 +87,7 @@ static kvzip_status score_passes(int passes, kvzip_dtype dt, const void* q, cons
   a.scale = scale;
   a.timeout_ns = g_timeout_ns.load();
   a.passes = passes;
+  a.sum_aggregation = sum_agg;
   a.test_stall = g_test_stall.load();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int launches = 0;
@@ -101,14 +102,14 @@ kvzip_status kvzip_score_chunk(kvzip_dtype dt, const void* q, const void* k_ctx,
                                const void* k_self, float* scores, int B, int G, int n_in,
                                int n_c, int d, float scale, void* workspace, size_t ws_bytes,
                                void* stream) {
-  return score_passes(3, dt, q, k_ctx, k_self, scores, B, G, n_in, n_c, d, scale, workspace,
+  return score_passes(3, 0, dt, q, k_ctx, k_self, scores, B, G, n_in, n_c, d, scale, workspace,
                       ws_bytes, stream);
 }
 
 kvzip_status kvzip_score_lse(kvzip_dtype dt, const void* q, const void* k_ctx,
                              const void* k_self, float* scores, int B, int G, int n_in, int n_c,
                              int d, float scale, void* workspace, size_t ws_bytes, void* stream) {
-  return score_passes(1, dt, q, k_ctx, k_self, scores, B, G, n_in, n_c, d, scale, workspace,
+  return score_passes(1, 0, dt, q, k_ctx, k_self, scores, B, G, n_in, n_c, d, scale, workspace,
                       ws_bytes, stream);
 }
 
@@ -116,8 +117,15 @@ kvzip_status kvzip_score_colmax(kvzip_dtype dt, const void* q, const void* k_ctx
                                 const void* k_self, float* scores, int B, int G, int n_in,
                                 int n_c, int d, float scale, void* workspace, size_t ws_bytes,
                                 void* stream) {
-  return score_passes(2, dt, q, k_ctx, k_self, scores, B, G, n_in, n_c, d, scale, workspace,
+  return score_passes(2, 0, dt, q, k_ctx, k_self, scores, B, G, n_in, n_c, d, scale, workspace,
                       ws_bytes, stream);
+}
+
+kvzip_status kvzip_score_chunk_sum(const void* q, const void* k_ctx, const void* k_self,
+                                   float* scores, int B, int G, int n_in, int n_c, int d,
+                                   float scale, void* workspace, size_t ws_bytes, void* stream) {
+  return score_passes(3, 1, KVZIP_BF16, q, k_ctx, k_self, scores, B, G, n_in, n_c, d, scale,
+                      workspace, ws_bytes, stream);
 }
 
 kvzip_status kvzip_workspace_status(void* workspace, void* stream) {
@@ -265,6 +273,64 @@ kvzip_status kvzip_decode_attention(const void* q, const void* k_packed, const v
   a.timeout_ns = g_timeout_ns.load();
   int launches = 0;
   cudaError_t e = kvzip::launch_decode(a, static_cast<cudaStream_t>(stream), &launches);
+  if (e == cudaSuccess) g_last_launches.store(launches);
+  return from_cuda(e);
+}
+
+kvzip_status kvzip_token_scores(const float* scores, int64_t n_heads, int64_t n_c,
+                                float* token_scores, void* stream) {
+  if (n_heads <= 0 || n_c <= 0 || n_heads * n_c >= (int64_t{1} << 31)) return KVZIP_ERR_INVALID_ARG;
+  if (!scores || !token_scores || !aligned(scores, 4) || !aligned(token_scores, 4))
+    return KVZIP_ERR_INVALID_ARG;
+  int launches = 0;
+  cudaError_t e = kvzip::launch_token_scores(scores, n_heads, n_c, token_scores,
+                                             static_cast<cudaStream_t>(stream), &launches);
+  if (e == cudaSuccess) g_last_launches.store(launches);
+  return from_cuda(e);
+}
+
+kvzip_status kvzip_expand_keep(const uint8_t* keep_pos, const int64_t* pos_offsets,
+                               int64_t n_heads, int64_t n_c, uint8_t* keep, int64_t* offsets,
+                               void* stream) {
+  if (n_heads <= 0 || n_c <= 0 || n_heads * n_c >= (int64_t{1} << 31)) return KVZIP_ERR_INVALID_ARG;
+  if (!keep_pos || !pos_offsets || !keep || !offsets || !aligned(pos_offsets, 8) ||
+      !aligned(offsets, 8))
+    return KVZIP_ERR_INVALID_ARG;
+  int launches = 0;
+  cudaError_t e = kvzip::launch_expand_keep(keep_pos, pos_offsets, n_heads, n_c, keep, offsets,
+                                            static_cast<cudaStream_t>(stream), &launches);
+  if (e == cudaSuccess) g_last_launches.store(launches);
+  return from_cuda(e);
+}
+
+size_t kvzip_select_per_head_workspace_size(int64_t n_heads, int64_t n_c) {
+  if (n_heads <= 0 || n_c < 0) return 0;
+  return kvzip::select_per_head_ws_bytes(n_heads, n_c);
+}
+
+kvzip_status kvzip_select_per_head(const float* scores, int64_t n_heads, int64_t n_c,
+                                   int64_t k_per_head, uint8_t* keep, int64_t* offsets,
+                                   void* workspace, size_t ws_bytes, void* stream) {
+  if (n_heads <= 0 || n_heads > 65535 || n_c <= 0 || k_per_head < 0 || k_per_head > n_c)
+    return KVZIP_ERR_INVALID_ARG;
+  if (n_heads * n_c >= (int64_t{1} << 31)) return KVZIP_ERR_INVALID_ARG;
+  if (!scores || !keep || !offsets || !workspace) return KVZIP_ERR_INVALID_ARG;
+  if (!aligned(scores, 16) || !aligned(offsets, 8) || !aligned(workspace, 256))
+    return KVZIP_ERR_INVALID_ARG;
+  if (ws_bytes < kvzip_select_per_head_workspace_size(n_heads, n_c)) return KVZIP_ERR_INVALID_ARG;
+  kvzip::SelectArgs a;
+  a.scores = scores;
+  a.N = n_heads * n_c;
+  a.k = k_per_head;
+  a.n_heads = n_heads;
+  a.n_c = n_c;
+  a.keep = keep;
+  a.offsets = offsets;
+  a.threshold = nullptr;
+  a.ws = workspace;
+  a.ws_bytes = ws_bytes;
+  int launches = 0;
+  cudaError_t e = kvzip::launch_select_per_head(a, static_cast<cudaStream_t>(stream), &launches);
   if (e == cudaSuccess) g_last_launches.store(launches);
   return from_cuda(e);
 }

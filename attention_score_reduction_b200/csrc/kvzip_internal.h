@@ -31,6 +31,7 @@ struct ScoreArgs {
   uint64_t timeout_ns;
   int passes;         // bit 0: pass 1 (row log-sum-exp), bit 1: pass 2 (column max)
   int test_stall;     // tensor-core scorer only: loader issues nothing (timeout tests)
+  int sum_aggregation = 0;  // pass 2 adds column sums instead of taking maxima
 };
 
 // Tensor-core (tcgen05) scorer for bf16 inputs.  Returns a cudaError_t.
@@ -48,6 +49,9 @@ struct SelectArgs {
   size_t ws_bytes;
 };
 size_t select_ws_bytes(int64_t N, int64_t n_heads);
+// Uniform head budgets: SelectArgs.k is the budget of every head.
+size_t select_per_head_ws_bytes(int64_t n_heads, int64_t n_c);
+cudaError_t launch_select_per_head(const SelectArgs& a, cudaStream_t s, int* launches);
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launches);
 
 struct CompactArgs {
@@ -65,6 +69,13 @@ struct CompactArgs {
 };
 size_t compact_ws_bytes(int64_t n_heads, int n_c);
 cudaError_t launch_compact(const CompactArgs& a, cudaStream_t s, int* launches);
+
+// Token-level scores and position-mask expansion.
+cudaError_t launch_token_scores(const float* scores, int64_t n_heads, int64_t n_c, float* tok,
+                                cudaStream_t s, int* launches);
+cudaError_t launch_expand_keep(const uint8_t* keep_pos, const int64_t* pos_off, int64_t n_heads,
+                               int64_t n_c, uint8_t* keep, int64_t* offsets, cudaStream_t s,
+                               int* launches);
 
 // Head-level scores: out[h] = max_j scores[h][j].
 cudaError_t launch_head_scores(const float* scores, int64_t n_heads, int64_t n_c, float* out,

@@ -180,7 +180,9 @@ struct TcParams {
   int test_stall;     // test hook: the loader issues no copies, so every wait runs out
 };
 
-template <int D, bool PASS2>
+// SUM (pass 2 only): column sums of the probabilities instead of maxima (the
+// rebuttal's average-aggregation ablation; sum and average rank identically).
+template <int D, bool PASS2, bool SUM = false>
 __global__ void __launch_bounds__(kThreads, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap bmap0,
                     const __grid_constant__ CUtensorMap bmap1, const TcParams p) {
@@ -440,7 +442,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         // ---------------- pass 2: running max over query rows of c*s - lse2
-        float best = -INFINITY;
+        // (or, for SUM, the running sum of 2^(c*s - lse2))
+        float best = SUM ? 0.f : -INFINITY;
 #pragma unroll 1
         for (int it = par; it < n_b; it += 2) {
           const int st = it % STAGES;
@@ -459,23 +462,36 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc_fence_before();
               mbar_arrive(&s_empty[t * 2 + par]);
             }
-            float b0 = best, b1 = -INFINITY;
+            if (SUM) {
+              float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int j = 0; j < CH; j += 4) {
-              const float4 L = L4[(ch + j) / 4];   // same address in every lane: broadcast
-              b0 = fmax3(b0, fmaf(v[j + 0], c, -L.x), fmaf(v[j + 1], c, -L.y));
-              b1 = fmax3(b1, fmaf(v[j + 2], c, -L.z), fmaf(v[j + 3], c, -L.w));
+              for (int j = 0; j < CH; j += 4) {
+                const float4 L = L4[(ch + j) / 4];
+                a0 += ex2_approx(fmaf(v[j + 0], c, -L.x)) + ex2_approx(fmaf(v[j + 1], c, -L.y));
+                a1 += ex2_approx(fmaf(v[j + 2], c, -L.z)) + ex2_approx(fmaf(v[j + 3], c, -L.w));
+              }
+              best += a0 + a1;
+            } else {
+              float b0 = best, b1 = -INFINITY;
+#pragma unroll
+              for (int j = 0; j < CH; j += 4) {
+                const float4 L = L4[(ch + j) / 4];   // same address in every lane: broadcast
+                b0 = fmax3(b0, fmaf(v[j + 0], c, -L.x), fmaf(v[j + 1], c, -L.y));
+                b1 = fmax3(b1, fmaf(v[j + 2], c, -L.z), fmaf(v[j + 3], c, -L.w));
+              }
+              best = fmaxf(b0, b1);
             }
-            best = fmaxf(b0, b1);
           }
           mbar_arrive(&l_empty[st]);
         }
         if (par == 1) xchg->x = best;
         named_barrier_sync(1 + t, 2 * kBM);
         if (par == 0 && !*abort_flag && arow < p.n_c) {
-          const float bb = fmaxf(best, xchg->x);
           float* dst = p.scores + static_cast<size_t>(b) * p.n_c + arow;
-          *dst = fmaxf(*dst, ex2_approx(bb));
+          if (SUM)
+            *dst += best + xchg->x;
+          else
+            *dst = fmaxf(*dst, ex2_approx(fmaxf(best, xchg->x)));
         }
       }
     } else if (!PASS2 && par == 0) {
@@ -547,6 +563,9 @@ static cudaError_t launch_tc(const ScoreArgs& a, cudaStream_t s, int* launches) 
   e = cudaFuncSetAttribute(score_tc_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Lay::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(score_tc_kernel<D, true, true>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM_ALLOC);
+  if (e != cudaSuccess) return e;
   // B operands only: A rows go straight from global memory into TMEM.
   CUtensorMap kmap, smap;
   if (!make_map(&kmap, a.k_ctx, a.B, a.n_c, D, Lay::BN) ||
@@ -580,7 +599,10 @@ static cudaError_t launch_tc(const ScoreArgs& a, cudaStream_t s, int* launches) 
   if (!make_map(&qmapB, a.q, a.B, a.R, D, Lay::BN)) return cudaErrorInvalidValue;
   p.a_ptr = static_cast<const uint16_t*>(a.k_ctx);
   dim3 g2((a.n_c + kATiles * kBM - 1) / (kATiles * kBM), a.B);
-  score_tc_kernel<D, true><<<g2, kThreads, Lay::SMEM_ALLOC, s>>>(qmapB, qmapB, p);
+  if (a.sum_aggregation)
+    score_tc_kernel<D, true, true><<<g2, kThreads, Lay::SMEM_ALLOC, s>>>(qmapB, qmapB, p);
+  else
+    score_tc_kernel<D, true><<<g2, kThreads, Lay::SMEM_ALLOC, s>>>(qmapB, qmapB, p);
   e = cudaGetLastError();
   if (e == cudaSuccess && launches) *launches += 1;
   return e;

@@ -8,7 +8,7 @@
 //
 // Scores are finite and >= 0, so their IEEE bit patterns, read as uint32, sort
 // like the values.  The threshold tau (the k-th largest bit pattern) is found
-// by a three-round radix select on 11 + 11 + 10 bits; every round is one
+// by a three-round radix select on 13 + 10 + 9 bits; every round is one
 // histogram pass over HBM plus a one-block pick, all on the stream with no
 // host round trip.  A mask pass then writes keep[f] and per-block kept counts;
 // a one-block scan turns those into per-head offsets.  When more elements equal
@@ -51,14 +51,17 @@ struct SelWs {
   uint32_t* blk_eq;   // equal-to-tau per mask block, scanned in place
 };
 
-// Radix rounds: bins, shift of the digit, bits fixed before the round, histogram offset.
-__host__ __device__ constexpr int hist_bins(int p) { return p == 2 ? 1024 : 2048; }
-__host__ __device__ constexpr int hist_shift(int p) { return p == 0 ? 21 : (p == 1 ? 10 : 0); }
+// Radix rounds of 13 + 10 + 9 bits: bins, shift of the digit, bits fixed before
+// the round, histogram offset.  Scores in (0, 1] share few exponents, so the
+// first round takes 5 mantissa bits along with sign and exponent to spread
+// them over enough shared-memory bins to keep atomic contention low.
+__host__ __device__ constexpr int hist_bins(int p) { return p == 0 ? 8192 : (p == 1 ? 1024 : 512); }
+__host__ __device__ constexpr int hist_shift(int p) { return p == 0 ? 19 : (p == 1 ? 9 : 0); }
 __host__ __device__ constexpr uint32_t hist_mask(int p) {
-  return p == 0 ? 0u : (p == 1 ? 0xFFE00000u : 0xFFFFFC00u);
+  return p == 0 ? 0u : (p == 1 ? 0xFFF80000u : 0xFFFFFE00u);
 }
-__host__ __device__ constexpr int hist_off(int p) { return p * 2048; }
-constexpr int kHistTotal = 5120;
+__host__ __device__ constexpr int hist_off(int p) { return p == 0 ? 0 : (p == 1 ? 8192 : 9216); }
+constexpr int kHistTotal = 9728;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -66,7 +69,11 @@ __host__ __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { retur
 
 int64_t segs_per_head(int64_t n_c) { return (n_c + kSelSeg - 1) / kSelSeg; }
 
+// One block per selection problem (the whole array, or one head for uniform
+// budgets): zero its histograms and set its state.
 __global__ void sel_init(SelState* st, uint32_t* hist, unsigned long long k, float* threshold) {
+  st += blockIdx.x;
+  hist += static_cast<size_t>(blockIdx.x) * kHistTotal;
   for (int i = threadIdx.x; i < kHistTotal; i += blockDim.x) hist[i] = 0;
   if (threadIdx.x == 0) {
     if (k == 0 && threshold) *threshold = INFINITY;
@@ -80,6 +87,7 @@ __global__ void sel_init(SelState* st, uint32_t* hist, unsigned long long k, flo
   }
 }
 
+// blockIdx.y selects the problem: elements [y * N, (y + 1) * N).
 template <int PASS>
 __global__ void __launch_bounds__(kHistThreads)
     sel_hist(const float* __restrict__ s, int64_t N, const SelState* st, uint32_t* hist) {
@@ -87,10 +95,14 @@ __global__ void __launch_bounds__(kHistThreads)
   constexpr int SH = hist_shift(PASS);
   constexpr uint32_t PM = hist_mask(PASS);
   __shared__ uint32_t h[NB];
+  s += static_cast<size_t>(blockIdx.y) * N;
+  st += blockIdx.y;
+  hist += static_cast<size_t>(blockIdx.y) * kHistTotal;
   for (int i = threadIdx.x; i < NB; i += blockDim.x) h[i] = 0;
   __syncthreads();
   const uint32_t prefix = st->prefix;
-  const int64_t n4 = N / 4;
+  // vector loads need 16-byte aligned problems (N a multiple of 4)
+  const int64_t n4 = (gridDim.y == 1 || N % 4 == 0) ? N / 4 : 0;
   const uint4* s4 = reinterpret_cast<const uint4*>(s);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
@@ -141,10 +153,12 @@ template <int PASS>
 __global__ void __launch_bounds__(kPickThreads)
     sel_pick(SelState* st, const uint32_t* hist, float* threshold) {
   constexpr int NB = hist_bins(PASS);
-  constexpr int PER = NB / kPickThreads;  // 2 or 1 bins per thread
+  constexpr int PER = (NB + kPickThreads - 1) / kPickThreads;  // 8, 1 or 1 bins per thread
   __shared__ unsigned long long sm[32];
   __shared__ int found_bin;
   __shared__ unsigned long long found_above;
+  st += blockIdx.x;                     // one block per selection problem
+  hist += static_cast<size_t>(blockIdx.x) * kHistTotal;
   if (st->keep_none) return;
   const uint32_t* h = hist + hist_off(PASS);
   // thread t owns bins NB-1-PER*t ... NB-PER*(t+1) (descending)
@@ -152,7 +166,8 @@ __global__ void __launch_bounds__(kPickThreads)
   uint32_t cnt[PER];
 #pragma unroll
   for (int j = 0; j < PER; ++j) {
-    cnt[j] = h[NB - 1 - (PER * threadIdx.x + j)];
+    const int bin = NB - 1 - (PER * static_cast<int>(threadIdx.x) + j);
+    cnt[j] = bin >= 0 ? h[bin] : 0u;
     mine += cnt[j];
   }
   const unsigned long long incl = block_incl_scan(mine, sm);
@@ -196,10 +211,11 @@ __device__ __forceinline__ uint32_t warp_excl_prefix(bool flag, uint32_t* total)
 // Count scores equal to tau per mask block (only when ties must be ranked).
 __global__ void __launch_bounds__(kSelThreads)
     sel_eqcount(const float* __restrict__ s, int64_t n_c, int64_t segs, const SelState* st,
-                uint32_t* blk_eq) {
-  if (st->keep_none || st->take_eq == st->n_eq) return;
+                uint32_t* blk_eq, int per_head) {
   const int64_t blk = blockIdx.x;
   const int64_t h = blk / segs, sg = blk % segs;
+  if (per_head) st += h;
+  if (st->keep_none || st->take_eq == st->n_eq) return;
   const int64_t j0 = sg * kSelSeg, j1 = imin64(j0 + kSelSeg, n_c);
   const float* base = s + h * n_c;
   const uint32_t tau = st->tau;
@@ -220,6 +236,9 @@ __global__ void __launch_bounds__(kSelThreads)
 // Exclusive scan of per-block values, in place, one block.
 __global__ void __launch_bounds__(kPickThreads)
     sel_scan_blocks(uint32_t* v, int64_t n, const SelState* st, int only_if_ties) {
+  // one block per selection problem: values [x * n, (x + 1) * n)
+  v += static_cast<size_t>(blockIdx.x) * n;
+  st += blockIdx.x;
   if (only_if_ties && (st->keep_none || st->take_eq == st->n_eq)) return;
   __shared__ unsigned long long sm[32];
   __shared__ unsigned long long carry;
@@ -240,9 +259,10 @@ __global__ void __launch_bounds__(kPickThreads)
 // keep[f] and kept count per block.
 __global__ void __launch_bounds__(kSelThreads)
     sel_mask(const float* __restrict__ s, int64_t n_c, int64_t segs, const SelState* st,
-             const uint32_t* blk_eq_base, uint8_t* keep, uint32_t* blk_cnt) {
+             const uint32_t* blk_eq_base, uint8_t* keep, uint32_t* blk_cnt, int per_head) {
   const int64_t blk = blockIdx.x;
   const int64_t h = blk / segs, sg = blk % segs;
+  if (per_head) st += h;
   const int64_t j0 = sg * kSelSeg, j1 = imin64(j0 + kSelSeg, n_c);
   const float* base = s + h * n_c;
   uint8_t* kb = keep + h * n_c;
@@ -328,6 +348,14 @@ SelWs carve(void* ws, int64_t nblk) {
 
 }  // namespace
 
+// Per-head (uniform budget) workspace: one state and one set of histograms per head.
+size_t per_head_ws_bytes(int64_t n_heads, int64_t n_c) {
+  const int64_t nblk = n_heads * segs_per_head(n_c);
+  return align_up(static_cast<size_t>(n_heads) * sizeof(SelState), 256) +
+         align_up(static_cast<size_t>(n_heads) * kHistTotal * 4, 256) +
+         2 * align_up(static_cast<size_t>(nblk) * 4, 256);
+}
+
 size_t select_ws_bytes(int64_t N, int64_t n_heads) {
   const int64_t n_c = n_heads > 0 ? N / n_heads : 0;
   const int64_t nblk = n_heads * segs_per_head(n_c);
@@ -354,13 +382,60 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launches) {
     sel_hist<2><<<grid, kHistThreads, 0, s>>>(a.scores, a.N, w.st, w.hist);
     sel_pick<2><<<1, kPickThreads, 0, s>>>(w.st, w.hist, a.threshold);
     sel_eqcount<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs, w.st,
-                                                                   w.blk_eq);
+                                                                   w.blk_eq, 0);
     sel_scan_blocks<<<1, kPickThreads, 0, s>>>(w.blk_eq, nblk, w.st, 1);
     n += 8;
   }
   sel_mask<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs, w.st,
-                                                              w.blk_eq, a.keep, w.blk_cnt);
+                                                              w.blk_eq, a.keep, w.blk_cnt, 0);
   sel_offsets<<<1, kPickThreads, 0, s>>>(w.blk_cnt, a.n_heads, segs, a.offsets);
+  n += 2;
+  if (launches) *launches += n;
+  return cudaGetLastError();
+}
+
+size_t select_per_head_ws_bytes(int64_t n_heads, int64_t n_c) {
+  return per_head_ws_bytes(n_heads, n_c);
+}
+
+// Uniform head budgets: the same radix selection run for every head at once
+// (grid dimension = head), k_per_head pairs kept in each.
+cudaError_t launch_select_per_head(const SelectArgs& a, cudaStream_t s, int* launches) {
+  const int64_t segs = segs_per_head(a.n_c);
+  const int64_t nblk = a.n_heads * segs;
+  uint8_t* p = static_cast<uint8_t*>(a.ws);
+  SelState* st = reinterpret_cast<SelState*>(p);
+  p += align_up(static_cast<size_t>(a.n_heads) * sizeof(SelState), 256);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(p);
+  p += align_up(static_cast<size_t>(a.n_heads) * kHistTotal * 4, 256);
+  uint32_t* blk_cnt = reinterpret_cast<uint32_t*>(p);
+  p += align_up(static_cast<size_t>(nblk) * 4, 256);
+  uint32_t* blk_eq = reinterpret_cast<uint32_t*>(p);
+  const unsigned H = static_cast<unsigned>(a.n_heads);
+  int n = 0;
+  sel_init<<<H, 1024, 0, s>>>(st, hist, static_cast<unsigned long long>(a.k), nullptr);
+  ++n;
+  if (a.k > 0) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t want = (a.n_c / 4 + kHistThreads - 1) / kHistThreads;
+    const int64_t cap = std::max<int64_t>(1, 4LL * sms / a.n_heads);
+    const dim3 grid(static_cast<unsigned>(std::max<int64_t>(1, std::min(want, cap))), H);
+    sel_hist<0><<<grid, kHistThreads, 0, s>>>(a.scores, a.n_c, st, hist);
+    sel_pick<0><<<H, kPickThreads, 0, s>>>(st, hist, nullptr);
+    sel_hist<1><<<grid, kHistThreads, 0, s>>>(a.scores, a.n_c, st, hist);
+    sel_pick<1><<<H, kPickThreads, 0, s>>>(st, hist, nullptr);
+    sel_hist<2><<<grid, kHistThreads, 0, s>>>(a.scores, a.n_c, st, hist);
+    sel_pick<2><<<H, kPickThreads, 0, s>>>(st, hist, nullptr);
+    sel_eqcount<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs, st,
+                                                                   blk_eq, 1);
+    sel_scan_blocks<<<H, kPickThreads, 0, s>>>(blk_eq, segs, st, 1);
+    n += 8;
+  }
+  sel_mask<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs, st, blk_eq,
+                                                              a.keep, blk_cnt, 1);
+  sel_offsets<<<1, kPickThreads, 0, s>>>(blk_cnt, a.n_heads, segs, a.offsets);
   n += 2;
   if (launches) *launches += n;
   return cudaGetLastError();

@@ -47,6 +47,11 @@ def _load() -> ctypes.CDLL:
         "kvzip_compact_workspace_size": (sz, [i64, i32]),
         "kvzip_compact": (i32, [vp, vp, vp, vp, i64, i32, i32, vp, vp, vp, vp, sz, vp]),
         "kvzip_head_scores": (i32, [vp, i64, i64, vp, vp]),
+        "kvzip_score_chunk_sum": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, sz, vp]),
+        "kvzip_token_scores": (i32, [vp, i64, i64, vp, vp]),
+        "kvzip_expand_keep": (i32, [vp, vp, i64, i64, vp, vp, vp]),
+        "kvzip_select_per_head_workspace_size": (sz, [i64, i64]),
+        "kvzip_select_per_head": (i32, [vp, i64, i64, i64, vp, vp, vp, sz, vp]),
         "kvzip_decode_workspace_size": (sz, [i64, i32, i32]),
         "kvzip_decode_attention": (i32, [vp, vp, vp, vp, i64, i32, i32, f32, vp, vp, sz, vp]),
         "kvzip_last_launch_count": (i32, []),
@@ -229,6 +234,60 @@ def compact(k: torch.Tensor, v: torch.Tensor, keep: torch.Tensor, offsets: torch
                            workspace.numel(), _stream(stream))
     _check(s, "kvzip_compact")
     return k_out, v_out, pos_out
+
+
+# ---------------------------------------------------------------- variants
+
+def score_chunk_sum(q, k_ctx, k_self, scores, workspace=None, scale: float = 0.0, stream=None):
+    """scores += per-key sums over query rows of the chunk's softmax (bf16 only)."""
+    for n, t in (("q", q), ("k_ctx", k_ctx), ("k_self", k_self)):
+        _dev_contig(n, t, torch.bfloat16)
+    _dev_contig("scores", scores, torch.float32)
+    B, G, n_in, d = q.shape
+    n_c = k_ctx.shape[1]
+    if workspace is None:
+        workspace = new_score_workspace(B, G, n_in, q.device)
+    _check(_lib.kvzip_score_chunk_sum(_ptr(q), _ptr(k_ctx), _ptr(k_self), _ptr(scores), B, G,
+                                      n_in, n_c, d, float(scale), _ptr(workspace),
+                                      workspace.numel(), _stream(stream)),
+           "kvzip_score_chunk_sum")
+    return scores
+
+
+def token_scores(scores: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+    """max over heads per position; scores [n_heads][n_c] float32 -> [n_c]."""
+    _dev_contig("scores", scores, torch.float32)
+    n_heads, n_c = scores.shape
+    out = torch.empty(n_c, dtype=torch.float32, device=scores.device) if out is None else out
+    _check(_lib.kvzip_token_scores(_ptr(scores), n_heads, n_c, _ptr(out), _stream(stream)),
+           "kvzip_token_scores")
+    return out
+
+
+def expand_keep(keep_pos: torch.Tensor, pos_offsets: torch.Tensor, n_heads: int, stream=None):
+    """Position mask (from select with n_heads = 1) -> per-head mask and offsets."""
+    n_c = keep_pos.numel()
+    keep = torch.empty(n_heads * n_c, dtype=torch.uint8, device=keep_pos.device)
+    offsets = torch.empty(n_heads + 1, dtype=torch.int64, device=keep_pos.device)
+    _check(_lib.kvzip_expand_keep(_ptr(keep_pos), _ptr(pos_offsets), n_heads, n_c, _ptr(keep),
+                                  _ptr(offsets), _stream(stream)), "kvzip_expand_keep")
+    return keep, offsets
+
+
+def select_per_head(scores: torch.Tensor, k_per_head: int, workspace=None, stream=None):
+    """Uniform budgets: top k_per_head of each head; scores [n_heads][n_c] float32."""
+    _dev_contig("scores", scores, torch.float32)
+    n_heads, n_c = scores.shape
+    dev = scores.device
+    keep = torch.empty(n_heads * n_c, dtype=torch.uint8, device=dev)
+    offsets = torch.empty(n_heads + 1, dtype=torch.int64, device=dev)
+    if workspace is None:
+        n = int(_lib.kvzip_select_per_head_workspace_size(n_heads, n_c))
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
+    _check(_lib.kvzip_select_per_head(_ptr(scores), n_heads, n_c, int(k_per_head), _ptr(keep),
+                                      _ptr(offsets), _ptr(workspace), workspace.numel(),
+                                      _stream(stream)), "kvzip_select_per_head")
+    return keep, offsets
 
 
 # ---------------------------------------------------------------- head scores

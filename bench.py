@@ -34,6 +34,13 @@ from attention_score_reduction_b200 import synth  # noqa: E402
 
 METRIC = "context tokens scored/sec (all layers+heads) @LLaMA3.1-8B 128K; % bf16 TC peak"
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per full launch of
+# each scorer pass on the 128K LLaMA3.1-8B workload, from an ncu capture of the
+# current kernels on one layer (8 units) scaled to the launch's 256 units (each
+# unit streams its own keys, so traffic grows with the units).
+NCU_TRAFFIC = {("llama8b_128k", 32, "score_pass1_lse"): 10.76e9,
+               ("llama8b_128k", 32, "score_pass2_colmax"): 9.51e9}
+
 
 def parse():
     ap = argparse.ArgumentParser()
@@ -268,7 +275,8 @@ def main():
     score_ms = (sum(p1) + sum(p2)) / args.steps
     executed_tf = (f1 + f2) * len(p1) / args.steps / (ms_per_step * 1e-3) / 1e12
     roofline = {"kernel": dominant, "bound": "tensor", "achieved": dom_tf, "peak": peak_tf,
-                "unit": "TFLOP/s", "frac": dom_tf / peak_tf, "traffic": None,
+                "unit": "TFLOP/s", "frac": dom_tf / peak_tf,
+                "traffic": NCU_TRAFFIC.get((wl.name, wl.L, dominant)),
                 "peak_source": f"{peaks['source']} bf16 sustained",
                 "flops_per_launch": dom_f}
     kernels = {

@@ -164,7 +164,7 @@ kvzip_status kvzip_select(const float* scores, int64_t N, int64_t k, int64_t n_h
  * library-owned static device array of 1 MiB on every GPU that loads the
  * library (held until the process exits).  It fits problems with
  * kvzip_select_workspace_size(N, n_heads) <= 1 MiB, i.e. roughly
- * n_heads * ceil(n_c / 8192) <= 128000 (all LLaMA3.1-8B / Qwen2.5-14B /
+ * n_heads * ceil(n_c / 8192) <= 126000 (all LLaMA3.1-8B / Qwen2.5-14B /
  * Gemma3-12B shapes up to 170K tokens); larger ones return
  * KVZIP_ERR_UNSUPPORTED without launching anything.  N must be >= 1.
  *   - The first call on each device looks up the array's device address with
@@ -226,6 +226,48 @@ kvzip_status kvzip_decode_attention(const void* q, const void* k_packed, const v
                                     const int64_t* offsets, int64_t n_heads, int G, int d,
                                     float scale, float* out, void* workspace, size_t ws_bytes,
                                     void* stream);
+
+/* ------------------------------------------------------------ variants */
+
+/*
+ * Sum aggregation (the rebuttal's average-aggregation ablation: sum and
+ * average give identical eviction priorities; max ranks better):
+ *   scores[b][j] += sum over query rows of softmax(...)[rho][j].
+ * Same arguments as kvzip_score_chunk without the dtype: bf16 inputs only.
+ * Zero `scores` before the first chunk.
+ */
+kvzip_status kvzip_score_chunk_sum(const void* q, const void* k_ctx, const void* k_self,
+                                   float* scores, int B, int G, int n_in, int n_c, int d,
+                                   float scale, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Token-level scores (blog post section 4.3.3): token_scores[j] = max over the
+ * n_heads = L*H heads of scores[h][j].  Select over them with kvzip_select
+ * (n_heads = 1) and turn the position mask into a per-head mask with
+ * kvzip_expand_keep.  Exact.
+ */
+kvzip_status kvzip_token_scores(const float* scores, int64_t n_heads, int64_t n_c,
+                                float* token_scores, void* stream);
+
+/* keep[h][j] = keep_pos[j] for every head; offsets[h] = h * kept positions,
+ * where kept positions = pos_offsets[1] - pos_offsets[0] (as kvzip_select with
+ * n_heads = 1 returns them; device memory). */
+kvzip_status kvzip_expand_keep(const uint8_t* keep_pos, const int64_t* pos_offsets,
+                               int64_t n_heads, int64_t n_c, uint8_t* keep, int64_t* offsets,
+                               void* stream);
+
+/* Bytes of workspace kvzip_select_per_head needs. */
+size_t kvzip_select_per_head_workspace_size(int64_t n_heads, int64_t n_c);
+
+/*
+ * Uniform head budgets (scime.ai summary, "Measured effects": worse than the
+ * non-uniform budgets a global ranking gives): keep the k_per_head largest
+ * scores inside every head, lower position first among equal scores.
+ * offsets[h] = h * k_per_head.  0 <= k_per_head <= n_c; scores 16-byte aligned.
+ */
+kvzip_status kvzip_select_per_head(const float* scores, int64_t n_heads, int64_t n_c,
+                                   int64_t k_per_head, uint8_t* keep, int64_t* offsets,
+                                   void* workspace, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------ head scores */
 
