@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-attention table")
+    ap.add_argument("--chunked", action="store_true",
+                    help="score chunk by chunk (pass 1 then pass 2) instead of the chunk pipeline")
     return ap.parse_args()
 
 
@@ -197,25 +199,43 @@ def main():
     torch.cuda.synchronize()
 
     stream = torch.cuda.current_stream()
-    per_chunk = []  # (ev0, ev1, ev2) per chunk, per timed step
+    per_launch = []  # (event before, event after, kernel name, flops) per scorer launch, timed steps
     stage_ev = []
+    C = len(chunks)
 
     def step(timed: bool):
         comp.reset()
         launches = 0
-        for q, ks in chunks:
+        n_sc = 2 * C if args.chunked else C + 1
+        for st in range(n_sc):
+            if args.chunked:   # per-chunk calls: pass 1 then pass 2 of chunk st // 2
+                q, ks = chunks[st // 2]
+                which = "lse" if st % 2 == 0 else "colmax"
+                f = bu.score_flops(wl.units, wl.G, q.shape[2], wl.n_c, wl.d)
+                name = "score_pass1_lse" if which == "lse" else "score_pass2_colmax"
+                flops = f["pass1"] if which == "lse" else f["pass2"]
+            else:              # pipeline: pass 1 of chunk st beside pass 2 of chunk st - 1
+                nxt = chunks[st] if st < C else None
+                prev = chunks[st - 1] if st > 0 else None
+                flops = 0.0
+                if nxt is not None:
+                    flops += bu.score_flops(wl.units, wl.G, nxt[0].shape[2], wl.n_c, wl.d)["pass1"]
+                if prev is not None:
+                    flops += bu.score_flops(wl.units, wl.G, prev[0].shape[2], wl.n_c,
+                                            wl.d)["pass2"]
+                name = ("score_pipelined" if nxt is not None and prev is not None else
+                        "score_pass1_lse" if nxt is not None else "score_pass2_colmax")
             if timed:
-                e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+                e0, e1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
                 e0.record(stream)
-            kz.score_chunk(q, k_ctx, ks, comp.scores, comp.score_ws, which="lse")
+            if args.chunked:
+                kz.score_chunk(q, k_ctx, ks, comp.scores, comp.score_ws, which=which)
+            else:
+                kz.score_pipeline_step(st, nxt, prev, k_ctx, comp.scores, comp.score_ws)
             launches += kz.last_launch_count()
             if timed:
                 e1.record(stream)
-            kz.score_chunk(q, k_ctx, ks, comp.scores, comp.score_ws, which="colmax")
-            launches += kz.last_launch_count()
-            if timed:
-                e2.record(stream)
-                per_chunk.append((e0, e1, e2, q.shape[2]))
+                per_launch.append((e0, e1, name, flops))
         if timed:
             s0, s1, s2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
             s0.record(stream)
@@ -254,34 +274,35 @@ def main():
     value = world * wl.n_c / (ms_per_step / 1e3)
 
     # per-kernel device times
-    p1 = [a.elapsed_time(b) for a, b, _, _ in per_chunk]
-    p2 = [b.elapsed_time(c) for _, b, c, _ in per_chunk]
+    peaks = bu.load_peaks(os.path.join(ROOT, "MEASURED_PEAKS.json"))
+    peak_tf = peaks["bf16_tflops_sustained"]
+    by_kernel = {}
+    for a, b, name, flops in per_launch:
+        by_kernel.setdefault(name, []).append((a.elapsed_time(b), flops))
+    kernels = {}
+    for name, rows in by_kernel.items():
+        t = sum(ms for ms, _ in rows) / len(rows)
+        f = sum(fl for _, fl in rows) / len(rows)
+        tf = f / (t * 1e-3) / 1e12
+        kernels[name] = {"launches_per_step": len(rows) // args.steps, "ms": t,
+                         "tflop_per_launch": f / 1e12, "tflops": tf, "frac_of_peak": tf / peak_tf}
+    dominant = max(by_kernel, key=lambda n: sum(ms for ms, _ in by_kernel[n]))
     sel = [a.elapsed_time(b) for a, b, _ in stage_ev]
     cmp = [b.elapsed_time(c) for _, b, c in stage_ev]
-    peaks = bu.load_peaks(os.path.join(ROOT, "MEASURED_PEAKS.json"))
-    fl = [bu.score_flops(wl.units, wl.G, n_in, wl.n_c, wl.d) for *_, n_in in per_chunk]
-    f1 = sum(f["pass1"] for f in fl) / len(fl)
-    f2 = sum(f["pass2"] for f in fl) / len(fl)
-    t1, t2 = sum(p1) / len(p1), sum(p2) / len(p2)
-    tf1, tf2 = f1 / (t1 * 1e-3) / 1e12, f2 / (t2 * 1e-3) / 1e12
-    peak_tf = peaks["bf16_tflops_sustained"]
-    dominant = "score_pass1_lse" if sum(p1) >= sum(p2) else "score_pass2_colmax"
-    dom_tf, dom_f = (tf1, f1) if dominant == "score_pass1_lse" else (tf2, f2)
     # selection / compaction bytes: scores read once + mask written; kept K and V rows
     # read and written once, positions written, mask read once.
     sel_bytes = N * 4 + N
     cmp_bytes = N + kept * wl.d * 2 * 2 * 2 + kept * 4
     t_sel, t_cmp = sum(sel) / len(sel), sum(cmp) / len(cmp)
-    score_ms = (sum(p1) + sum(p2)) / args.steps
-    executed_tf = (f1 + f2) * len(p1) / args.steps / (ms_per_step * 1e-3) / 1e12
-    roofline = {"kernel": dominant, "bound": "tensor", "achieved": dom_tf, "peak": peak_tf,
-                "unit": "TFLOP/s", "frac": dom_tf / peak_tf,
+    score_ms = sum(ms for rows in by_kernel.values() for ms, _ in rows) / args.steps
+    score_flops = sum(fl for rows in by_kernel.values() for _, fl in rows) / args.steps
+    dk = kernels[dominant]
+    roofline = {"kernel": dominant, "bound": "tensor", "achieved": dk["tflops"], "peak": peak_tf,
+                "unit": "TFLOP/s", "frac": dk["frac_of_peak"],
                 "traffic": NCU_TRAFFIC.get((wl.name, wl.L, dominant)),
                 "peak_source": f"{peaks['source']} bf16 sustained",
-                "flops_per_launch": dom_f}
-    kernels = {
-        "score_pass1_lse": {"ms": t1, "tflops": tf1, "frac_of_peak": tf1 / peak_tf},
-        "score_pass2_colmax": {"ms": t2, "tflops": tf2, "frac_of_peak": tf2 / peak_tf},
+                "flops_per_launch": dk["tflop_per_launch"] * 1e12}
+    kernels.update({
         "select": {"ms": t_sel, "gbs": sel_bytes / (t_sel * 1e-3) / 1e9,
                    "frac_of_hbm": sel_bytes / (t_sel * 1e-3) / 1e9 / peaks["hbm_gbs"]},
         "compact": {"ms": t_cmp, "gbs": cmp_bytes / (t_cmp * 1e-3) / 1e9,
@@ -289,10 +310,9 @@ def main():
         "select_plus_compact_frac_of_hbm":
             (sel_bytes + cmp_bytes) / ((t_sel + t_cmp) * 1e-3) / 1e9 / peaks["hbm_gbs"],
         "scoring_ms_per_step": score_ms,
-        "scoring_pct_bf16_tc_peak": 100.0 * (f1 + f2) * len(p1) / args.steps
-                                     / (score_ms * 1e-3) / 1e12 / peak_tf,
-        "step_pct_bf16_tc_peak": 100.0 * executed_tf / peak_tf,
-    }
+        "scoring_pct_bf16_tc_peak": 100.0 * score_flops / (score_ms * 1e-3) / 1e12 / peak_tf,
+        "step_pct_bf16_tc_peak": 100.0 * score_flops / (ms_per_step * 1e-3) / 1e12 / peak_tf,
+    })
 
     # ------------------------------------------------------------ decode over the kept cache
     decode = None
@@ -310,6 +330,7 @@ def main():
            "data": "synthetic", "config": config_dict(wl, r), "parallelism":
            f"{world} independent contexts, one per GPU", "clocks": clocks,
            "gpu_launches": launches, "roofline": roofline, "kernels": kernels,
+           "scoring": "per-chunk passes" if args.chunked else "chunk pipeline",
            "pct_bf16_tc_peak": kernels["step_pct_bf16_tc_peak"], "e2e": e2e,
            "decode_attention": decode}
 
