@@ -129,102 +129,7 @@ kvzip_status kvzip_score_chunk_sum(const void* q, const void* k_ctx, const void*
 }
 
 size_t kvzip_score_context_workspace_size(int B, int G, int max_n_in) {
-  if (B < 0 || G < 0 || max_n_in < 0) return 0;
-  const int64_t R = static_cast<int64_t>(G) * max_n_in;
-  return kvzip::kScoreWsHeader + 2 * static_cast<size_t>(B) * static_cast<size_t>(row_pad(R)) * 4;
-}
-
-kvzip_status kvzip_score_pipeline_step(kvzip_dtype dt, int step, const void* q_next,
-                                       const void* k_self_next, int n_in_next,
-                                       const void* q_prev, int n_in_prev, const void* k_ctx,
-                                       float* scores, int B, int G, int n_c, int d, float scale,
-                                       void* workspace, size_t ws_bytes, void* stream) {
-  if (dt != KVZIP_BF16 && dt != KVZIP_F32) return KVZIP_ERR_INVALID_ARG;
-  if (step < 0 || B < 0 || G < 0 || n_c < 0) return KVZIP_ERR_INVALID_ARG;
-  if (d != 128 && d != 256) return d > 0 ? KVZIP_ERR_UNSUPPORTED : KVZIP_ERR_INVALID_ARG;
-  if ((q_next && (!k_self_next || n_in_next <= 0)) || (q_prev && n_in_prev <= 0))
-    return KVZIP_ERR_INVALID_ARG;
-  if (B == 0 || G == 0 || n_c == 0 || (!q_next && !q_prev)) {
-    g_last_launches.store(0);
-    return KVZIP_OK;
-  }
-  if (!k_ctx || !scores || !workspace) return KVZIP_ERR_INVALID_ARG;
-  if (B > 65535) return KVZIP_ERR_UNSUPPORTED;
-  if ((q_next && (!aligned(q_next, 16) || !aligned(k_self_next, 16))) ||
-      (q_prev && !aligned(q_prev, 16)) || !aligned(k_ctx, 16) || !aligned(scores, 4) ||
-      !aligned(workspace, 256))
-    return KVZIP_ERR_INVALID_ARG;
-  if (ws_bytes < kvzip::kScoreWsHeader) return KVZIP_ERR_INVALID_ARG;
-  // two lse2 slots; chunk c uses slot c % 2 (written at step c, read at step c + 1)
-  const size_t slot_bytes = ((ws_bytes - kvzip::kScoreWsHeader) / 2) & ~static_cast<size_t>(255);
-  const int64_t R_next = q_next ? static_cast<int64_t>(G) * n_in_next : 0;
-  const int64_t R_prev = q_prev ? static_cast<int64_t>(G) * n_in_prev : 0;
-  if (R_next > INT_MAX - kvzip::kRowPad || R_prev > INT_MAX - kvzip::kRowPad)
-    return KVZIP_ERR_UNSUPPORTED;
-  if (static_cast<size_t>(B) * static_cast<size_t>(row_pad(R_next)) * 4 > slot_bytes ||
-      static_cast<size_t>(B) * static_cast<size_t>(row_pad(R_prev)) * 4 > slot_bytes)
-    return KVZIP_ERR_INVALID_ARG;
-  if (!(scale > 0.f) || std::isinf(scale)) scale = 1.0f / std::sqrt(static_cast<float>(d));
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  float* slot_next = reinterpret_cast<float*>(ws + kvzip::kScoreWsHeader + (step & 1) * slot_bytes);
-  float* slot_prev =
-      reinterpret_cast<float*>(ws + kvzip::kScoreWsHeader + ((step + 1) & 1) * slot_bytes);
-  uint32_t* status = static_cast<uint32_t*>(workspace);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int launches = 0;
-  cudaError_t e = cudaSuccess;
-  if (dt == KVZIP_BF16 && d == 128 && q_next && q_prev) {
-    kvzip::FusedArgs f{};
-    f.k_ctx = k_ctx;
-    f.scores = scores;
-    f.status = status;
-    f.B = B;
-    f.G = G;
-    f.n_c = n_c;
-    f.d = d;
-    f.scale = scale;
-    f.timeout_ns = g_timeout_ns.load();
-    f.test_stall = g_test_stall.load();
-    f.q1 = q_next;
-    f.k_self1 = k_self_next;
-    f.n_in1 = n_in_next;
-    f.lse_out = slot_next;
-    f.R_pad1 = static_cast<int>(row_pad(R_next));
-    f.q2 = q_prev;
-    f.n_in2 = n_in_prev;
-    f.lse_in = slot_prev;
-    f.R_pad2 = static_cast<int>(row_pad(R_prev));
-    e = kvzip::launch_score_fused(f, s, &launches);
-  } else {
-    // one pass at a time: pass 2 of the previous chunk, then pass 1 of the next
-    for (int half = 0; half < 2 && e == cudaSuccess; ++half) {
-      const void* q = half == 0 ? q_prev : q_next;
-      if (!q) continue;
-      kvzip::ScoreArgs a;
-      a.q = q;
-      a.k_ctx = k_ctx;
-      a.k_self = half == 0 ? k_ctx : k_self_next;   // pass 2 never reads self keys
-      a.scores = scores;
-      a.status = status;
-      a.lse2 = half == 0 ? slot_prev : slot_next;
-      a.B = B;
-      a.G = G;
-      a.n_in = half == 0 ? n_in_prev : n_in_next;
-      a.n_c = n_c;
-      a.d = d;
-      a.R = static_cast<int>(half == 0 ? R_prev : R_next);
-      a.R_pad = static_cast<int>(row_pad(a.R));
-      a.scale = scale;
-      a.timeout_ns = g_timeout_ns.load();
-      a.passes = half == 0 ? 2 : 1;
-      a.test_stall = g_test_stall.load();
-      e = (dt == KVZIP_BF16) ? kvzip::launch_score_tc(a, s, &launches)
-                             : kvzip::launch_score_simt_f32(a, s, &launches);
-    }
-  }
-  if (e == cudaErrorInvalidValue) return KVZIP_ERR_INVALID_ARG;  // tensor map rejected the layout
-  if (e == cudaSuccess) g_last_launches.store(launches);
-  return from_cuda(e);
+  return kvzip_score_workspace_size(B, G, max_n_in);
 }
 
 kvzip_status kvzip_score_context(kvzip_dtype dt, int n_chunks, const void* const* q,
@@ -233,15 +138,16 @@ kvzip_status kvzip_score_context(kvzip_dtype dt, int n_chunks, const void* const
                                  void* workspace, size_t ws_bytes, void* stream) {
   if (n_chunks < 0) return KVZIP_ERR_INVALID_ARG;
   if (n_chunks > 0 && (!q || !k_self || !n_in)) return KVZIP_ERR_INVALID_ARG;
-  for (int c = 0; c < n_chunks; ++c)
+  int max_n_in = 0;
+  for (int c = 0; c < n_chunks; ++c) {
     if (!q[c] || !k_self[c] || n_in[c] <= 0) return KVZIP_ERR_INVALID_ARG;
+    max_n_in = n_in[c] > max_n_in ? n_in[c] : max_n_in;
+  }
+  if (ws_bytes < kvzip_score_workspace_size(B, G, max_n_in)) return KVZIP_ERR_INVALID_ARG;
   int launches = 0;
-  for (int step = 0; step <= n_chunks && n_chunks > 0; ++step) {
-    const bool nx = step < n_chunks, pv = step > 0;
-    const kvzip_status st = kvzip_score_pipeline_step(
-        dt, step, nx ? q[step] : nullptr, nx ? k_self[step] : nullptr, nx ? n_in[step] : 0,
-        pv ? q[step - 1] : nullptr, pv ? n_in[step - 1] : 0, k_ctx, scores, B, G, n_c, d,
-        scale, workspace, ws_bytes, stream);
+  for (int c = 0; c < n_chunks; ++c) {
+    const kvzip_status st = score_passes(3, 0, dt, q[c], k_ctx, k_self[c], scores, B, G, n_in[c],
+                                         n_c, d, scale, workspace, ws_bytes, stream);
     if (st != KVZIP_OK) return st;
     launches += g_last_launches.load();
   }

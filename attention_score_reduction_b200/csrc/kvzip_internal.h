@@ -36,27 +36,6 @@ struct ScoreArgs {
 
 // Tensor-core (tcgen05) scorer for bf16 inputs.  Returns a cudaError_t.
 cudaError_t launch_score_tc(const ScoreArgs& a, cudaStream_t s, int* launches);
-// Chunk-pipelined tensor-core scorer (d = 128): pass 1 of one chunk and pass 2
-// of the previous chunk in one launch.  Either half may be absent (null q1 / q2).
-struct FusedArgs {
-  const void* k_ctx;
-  float* scores;
-  uint32_t* status;
-  int B, G, n_c, d;
-  float scale;
-  uint64_t timeout_ns;
-  int test_stall;
-  const void* q1;       // pass 1: queries [B][G*n_in1][d], self keys [B][n_in1][d]
-  const void* k_self1;
-  int n_in1;
-  float* lse_out;       // [B][R_pad1]
-  int R_pad1;
-  const void* q2;       // pass 2: queries [B][G*n_in2][d], normalisers [B][R_pad2]
-  int n_in2;
-  const float* lse_in;
-  int R_pad2;
-};
-cudaError_t launch_score_fused(const FusedArgs& a, cudaStream_t s, int* launches);
 // CUDA-core scorer for fp32 inputs.
 cudaError_t launch_score_simt_f32(const ScoreArgs& a, cudaStream_t s, int* launches);
 

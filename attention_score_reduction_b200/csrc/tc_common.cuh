@@ -81,21 +81,6 @@ __device__ __forceinline__ void tmem_ld_tile(uint32_t taddr, float (&v)[64]) { t
 __device__ __forceinline__ void tmem_ld_tile(uint32_t taddr, float (&v)[48]) { tmem_ld48(taddr, v); }
 __device__ __forceinline__ void tmem_ld_tile(uint32_t taddr, float (&v)[32]) { tmem_ld32(taddr, v); }
 
-// Barrier with an OR-reduction over the participating threads: every thread gets
-// the same answer, so a group of warps can agree to stop at the same item.
-__device__ __forceinline__ bool bar_red_or(int id, int count, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(count)
-      : "memory");
-  return r != 0;
-}
-
 // ------------------------------------------------------------------ host side
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,

@@ -39,8 +39,6 @@ def _load() -> ctypes.CDLL:
         "kvzip_score_lse": (i32, [i32, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, sz, vp]),
         "kvzip_score_colmax": (i32, [i32, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, sz, vp]),
         "kvzip_score_context_workspace_size": (sz, [i32, i32, i32]),
-        "kvzip_score_pipeline_step": (i32, [i32, i32, vp, vp, i32, vp, i32, vp, vp, i32, i32, i32,
-                                            i32, f32, vp, sz, vp]),
         "kvzip_score_context": (i32, [i32, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, vp,
                                       sz, vp]),
         "kvzip_workspace_status": (i32, [vp, vp]),
@@ -156,12 +154,12 @@ def context_workspace_size(B: int, G: int, max_n_in: int) -> int:
 
 
 def new_context_workspace(B: int, G: int, max_n_in: int, device=None) -> torch.Tensor:
-    """Zero-initialised workspace for the chunk pipeline (two normaliser slots)."""
+    """Zero-initialised workspace for score_context (status word + normalisers)."""
     n = context_workspace_size(B, G, max_n_in)
     return torch.zeros(max(n, 256), dtype=torch.uint8, device=device or "cuda")
 
 
-def _chunk_check(q, k_self, k_ctx, scores):
+def _chunk_check(q, k_self, k_ctx):
     _dev_contig("q", q, k_ctx.dtype)
     _dev_contig("k_self", k_self, k_ctx.dtype)
     B, G, n_in, d = q.shape
@@ -170,36 +168,11 @@ def _chunk_check(q, k_self, k_ctx, scores):
     return n_in
 
 
-def score_pipeline_step(step: int, nxt, prev, k_ctx: torch.Tensor, scores: torch.Tensor,
-                        workspace: torch.Tensor, scale: float = 0.0, stream=None):
-    """One step of the chunk pipeline (kvzip_score_pipeline_step): pass 1 of chunk
-    ``step`` (``nxt`` = (q, k_self) or None) and pass 2 of chunk ``step - 1``
-    (``prev`` = (q, k_self) or None) in one launch where the shape allows."""
-    _dev_contig("k_ctx", k_ctx)
-    _dev_contig("scores", scores, torch.float32)
-    B, n_c, d = k_ctx.shape
-    G = (nxt or prev)[0].shape[1] if (nxt or prev) else 1
-    qn = ksn = qp = None
-    n_in_n = n_in_p = 0
-    if nxt is not None:
-        qn, ksn = nxt
-        n_in_n = _chunk_check(qn, ksn, k_ctx, scores)
-    if prev is not None:
-        qp, ksp = prev
-        n_in_p = _chunk_check(qp, ksp, k_ctx, scores)
-    s = _lib.kvzip_score_pipeline_step(
-        _dtype_code(k_ctx), int(step), _ptr(qn), _ptr(ksn), n_in_n, _ptr(qp), n_in_p, _ptr(k_ctx),
-        _ptr(scores), B, G, n_c, d, float(scale), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _stream(stream))
-    _check(s, "kvzip_score_pipeline_step")
-    return scores
-
-
 def score_context(chunks, k_ctx: torch.Tensor, scores: torch.Tensor,
                   workspace: torch.Tensor | None = None, scale: float = 0.0, stream=None):
-    """Score every chunk of one context (kvzip_score_context): the same running
-    maximum as ``score_chunk`` over the chunks in order, with pass 1 of each chunk
-    sharing the GPU with pass 2 of the one before.  ``chunks`` = [(q, k_self), ...]."""
+    """Score every chunk of one context in one call (kvzip_score_context): the
+    same running maximum as ``score_chunk`` over the chunks in order.
+    ``chunks`` = [(q, k_self), ...] device tensors."""
     _dev_contig("k_ctx", k_ctx)
     _dev_contig("scores", scores, torch.float32)
     B, n_c, d = k_ctx.shape
@@ -209,7 +182,7 @@ def score_context(chunks, k_ctx: torch.Tensor, scores: torch.Tensor,
     if n == 0:
         return scores
     G = chunks[0][0].shape[1]
-    n_in = [_chunk_check(q, ks, k_ctx, scores) for q, ks in chunks]
+    n_in = [_chunk_check(q, ks, k_ctx) for q, ks in chunks]
     if any(q.shape[1] != G for q, _ in chunks):
         raise ValueError("every chunk must have the same number of query heads")
     if workspace is None:

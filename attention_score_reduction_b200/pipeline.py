@@ -4,10 +4,9 @@ selection and per-head compaction, through libkvzip.
 This is the user-facing call.  ``Compressor`` owns the device buffers for one
 context shape and runs the three C-ABI calls on a CUDA stream:
 
-  1. ``kvzip_score_pipeline_step`` once per reconstruction chunk plus once
-     more (blog post section 4.5: chunked scoring keeps memory linear in n_c),
-     merging into the L x H x n_c score tensor by a running max; each step runs
-     pass 1 of one chunk beside pass 2 of the chunk before it;
+  1. ``kvzip_score_context`` (all chunks) or ``kvzip_score_chunk`` once per
+     reconstruction chunk (blog post section 4.5: chunked scoring keeps memory
+     linear in n_c), merging into the L x H x n_c score tensor by a running max;
   2. ``kvzip_select`` once per context (scime.ai summary, "Approach": evict the
      lowest-scoring pairs once, query-agnostically), global over (l, h, j);
   3. ``kvzip_compact`` once, packing the kept K/V rows per head.
@@ -48,7 +47,6 @@ class Compressor:
         self.device = torch.device(device)
         N = units * n_c
         self.scores = torch.zeros(units, n_c, dtype=torch.float32, device=self.device)
-        # status word + two normaliser slots (also serves kvzip_score_chunk)
         self.score_ws = kz.new_context_workspace(units, G, max_n_in, self.device)
         self.select_ws = torch.empty(max(kz.select_workspace_size(N, units), 256),
                                      dtype=torch.uint8, device=self.device)
@@ -64,12 +62,6 @@ class Compressor:
 
     def score_chunk(self, q, k_ctx, k_self, scale: float = 0.0, stream=None):
         kz.score_chunk(q, k_ctx, k_self, self.scores, self.score_ws, scale, stream)
-        self.launches += kz.last_launch_count()
-
-    def score_step(self, step: int, nxt, prev, k_ctx, scale: float = 0.0, stream=None):
-        """Step ``step`` of the chunk pipeline: pass 1 of ``nxt`` = (q, k_self) of
-        chunk ``step`` beside pass 2 of ``prev``, chunk ``step - 1`` (either None)."""
-        kz.score_pipeline_step(step, nxt, prev, k_ctx, self.scores, self.score_ws, scale, stream)
         self.launches += kz.last_launch_count()
 
     def select(self, r: float, stream=None) -> int:
@@ -134,12 +126,9 @@ def compress_from_host(comp: Compressor, k_ctx_h, v_h, q_chunks_h, ks_chunks_h, 
             evs.append(e)
     comp.reset()
     main.wait_event(ev_kv)
-    chunks = list(zip(dev_bufs["q"], dev_bufs["ks"]))
-    for step in range(len(chunks) + 1):
-        if step < len(chunks):
-            main.wait_event(evs[step])
-        comp.score_step(step, chunks[step] if step < len(chunks) else None,
-                        chunks[step - 1] if step > 0 else None, dev_bufs["k_ctx"], scale)
+    for qd, ksd, e in zip(dev_bufs["q"], dev_bufs["ks"], evs):
+        main.wait_event(e)
+        comp.score_chunk(qd, dev_bufs["k_ctx"], ksd, scale)
     kept = comp.select(r)
     k_out, v_out, pos = comp.compact(dev_bufs["k_ctx"], dev_bufs["v"], kept)
     d2h = 0

@@ -57,8 +57,8 @@ def parse():
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-attention table")
-    ap.add_argument("--chunked", action="store_true",
-                    help="score chunk by chunk (pass 1 then pass 2) instead of the chunk pipeline")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the head-level / ablation kernel timings")
     return ap.parse_args()
 
 
@@ -201,41 +201,22 @@ def main():
     stream = torch.cuda.current_stream()
     per_launch = []  # (event before, event after, kernel name, flops) per scorer launch, timed steps
     stage_ev = []
-    C = len(chunks)
 
     def step(timed: bool):
         comp.reset()
         launches = 0
-        n_sc = 2 * C if args.chunked else C + 1
-        for st in range(n_sc):
-            if args.chunked:   # per-chunk calls: pass 1 then pass 2 of chunk st // 2
-                q, ks = chunks[st // 2]
-                which = "lse" if st % 2 == 0 else "colmax"
-                f = bu.score_flops(wl.units, wl.G, q.shape[2], wl.n_c, wl.d)
-                name = "score_pass1_lse" if which == "lse" else "score_pass2_colmax"
-                flops = f["pass1"] if which == "lse" else f["pass2"]
-            else:              # pipeline: pass 1 of chunk st beside pass 2 of chunk st - 1
-                nxt = chunks[st] if st < C else None
-                prev = chunks[st - 1] if st > 0 else None
-                flops = 0.0
-                if nxt is not None:
-                    flops += bu.score_flops(wl.units, wl.G, nxt[0].shape[2], wl.n_c, wl.d)["pass1"]
-                if prev is not None:
-                    flops += bu.score_flops(wl.units, wl.G, prev[0].shape[2], wl.n_c,
-                                            wl.d)["pass2"]
-                name = ("score_pipelined" if nxt is not None and prev is not None else
-                        "score_pass1_lse" if nxt is not None else "score_pass2_colmax")
-            if timed:
-                e0, e1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
-                e0.record(stream)
-            if args.chunked:
+        for q, ks in chunks:   # per chunk: pass 1 (row normalisers), then pass 2 (column max)
+            f = bu.score_flops(wl.units, wl.G, q.shape[2], wl.n_c, wl.d)
+            for which, name in (("lse", "score_pass1_lse"), ("colmax", "score_pass2_colmax")):
+                if timed:
+                    e0, e1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
+                    e0.record(stream)
                 kz.score_chunk(q, k_ctx, ks, comp.scores, comp.score_ws, which=which)
-            else:
-                kz.score_pipeline_step(st, nxt, prev, k_ctx, comp.scores, comp.score_ws)
-            launches += kz.last_launch_count()
-            if timed:
-                e1.record(stream)
-                per_launch.append((e0, e1, name, flops))
+                launches += kz.last_launch_count()
+                if timed:
+                    e1.record(stream)
+                    per_launch.append((e0, e1, name,
+                                       f["pass1"] if which == "lse" else f["pass2"]))
         if timed:
             s0, s1, s2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
             s0.record(stream)
@@ -319,6 +300,10 @@ def main():
     if not args.no_decode:
         decode = run_decode(wl, comp, k_ctx, v, dev, peaks)
 
+    variants = None
+    if not args.no_variants:
+        variants = run_variants(wl, comp, k_ctx, chunks[0], r, dev, peaks)
+
     # ------------------------------------------------------------ end to end
     e2e = None
     if not args.no_e2e:
@@ -330,9 +315,8 @@ def main():
            "data": "synthetic", "config": config_dict(wl, r), "parallelism":
            f"{world} independent contexts, one per GPU", "clocks": clocks,
            "gpu_launches": launches, "roofline": roofline, "kernels": kernels,
-           "scoring": "per-chunk passes" if args.chunked else "chunk pipeline",
            "pct_bf16_tc_peak": kernels["step_pct_bf16_tc_peak"], "e2e": e2e,
-           "decode_attention": decode}
+           "decode_attention": decode, "variants": variants}
 
     # free device memory before the CPU baseline allocates host buffers
     del chunks, k_ctx, v, comp
@@ -348,6 +332,67 @@ def main():
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+def _time_ms(fn, flush, iters=10, warm=3):
+    ms = 0.0
+    for i in range(iters + warm):
+        flush.fill_(i & 0xff)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= warm:
+            ms += e0.elapsed_time(e1)
+    return ms / iters
+
+
+def run_variants(wl, comp, k_ctx, chunk, r, dev, peaks):
+    """The ablation and head-level kernels on the bench workload's final scores.
+
+    head_scores and token_scores read the L x H x n_c scores once; expand_keep
+    writes the per-head mask from a position mask; select_per_head is the
+    uniform-budget selection (same bytes as the global one); score_chunk_sum is
+    the sum-aggregation pass 2 of one chunk (tensor cores).  L2 is flushed
+    before every timed launch.
+    """
+    from attention_score_reduction_b200 import kvzip as kz
+    units, n_c = wl.units, wl.n_c
+    N = units * n_c
+    S = comp.scores
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
+    hbm = peaks["hbm_gbs"]
+    out = {}
+
+    def bw(name, ms, nbytes):
+        g = nbytes / (ms * 1e-3) / 1e9
+        out[name] = {"ms": ms, "bytes": nbytes, "gbs": g, "frac_of_hbm": g / hbm}
+
+    hs = torch.empty(units, dtype=torch.float32, device=dev)
+    bw("head_scores", _time_ms(lambda: kz.head_scores(S, hs), flush), N * 4 + units * 4)
+    tok = torch.empty(n_c, dtype=torch.float32, device=dev)
+    bw("token_scores", _time_ms(lambda: kz.token_scores(S, tok), flush), N * 4 + n_c * 4)
+    kt = kz.keep_count(r, n_c)
+    keep_pos, pos_off, _ = kz.select(tok, kt, 1)
+    bw("expand_keep", _time_ms(lambda: kz.expand_keep(keep_pos, pos_off, units), flush),
+       n_c + N + (units + 1) * 8)
+    ws = torch.empty(max(int(kz.library().kvzip_select_per_head_workspace_size(units, n_c)), 256),
+                     dtype=torch.uint8, device=dev)
+    kph = kz.keep_count(r, n_c)
+    bw("select_per_head", _time_ms(lambda: kz.select_per_head(S, kph, ws), flush), N * 4 + N)
+    q, ks = chunk
+    tmp = torch.zeros_like(S)
+    sws = kz.new_score_workspace(units, wl.G, q.shape[2], dev)
+
+    # kvzip_score_chunk_sum runs both passes; timed whole against both passes' flops
+    ms = _time_ms(lambda: kz.score_chunk_sum(q, k_ctx, ks, tmp, sws), flush, iters=3, warm=1)
+    f = bu.score_flops(units, wl.G, q.shape[2], n_c, wl.d)
+    tf = (f["pass1"] + f["pass2"]) / (ms * 1e-3) / 1e12
+    out["score_chunk_sum"] = {"ms": ms, "tflop": (f["pass1"] + f["pass2"]) / 1e12, "tflops": tf,
+                              "frac_of_peak": tf / peaks["bf16_tflops_sustained"]}
+    del tmp
+    return out
 
 
 def run_decode(wl, comp, k_ctx, v, dev, peaks, ratios=(1.0, 0.8, 0.6, 0.4, 0.2), iters=20):

@@ -106,40 +106,24 @@ kvzip_status kvzip_score_colmax(kvzip_dtype dt, const void* q, const void* k_ctx
                                 void* stream);
 
 /*
- * Multi-chunk scoring (all reconstruction chunks of one context in one call).
- * The chunks of the blog post's section 4.5 are scored one after another
- * into the same running maximum; pass 2 of chunk c needs only chunk c's row
- * normalisers, so pass 1 of chunk c+1 can run beside it.  With bf16 and
- * d = 128 each step after the first is ONE kernel launch doing both (pass 1
- * of chunk c+1 is bound by the exponentials, pass 2 of chunk c by the tensor
- * cores); other shapes run the two passes back to back.
+ * Multi-chunk scoring: all reconstruction chunks of one context in one call
+ * (blog post section 4.5: the context is reconstructed chunk by chunk and
+ * the chunk scores are merged by a running maximum).  Equivalent to
+ * kvzip_score_chunk for chunk 0, 1, ..., n_chunks-1 in order on one stream
+ * and workspace; each chunk is two kernel launches (row normalisers, then
+ * column maxima).
  *
- * Workspace: kvzip_score_context_workspace_size(B, G, max_n_in) bytes,
- * 256-byte aligned, zeroed before first use: the status word (as for
- * kvzip_score_chunk) and two normaliser slots; chunk c uses slot c % 2.
- * Each slot is (ws_bytes - 256) / 2 bytes rounded down to a multiple of 256
- * and must hold B * G * n_in (rows padded to 768) floats of every chunk.
+ *   q, k_self, n_in  HOST arrays of n_chunks entries: device pointers to chunk
+ *                    c's queries [B][G][n_in[c]][d] and self keys
+ *                    [B][n_in[c]][d], and its row count n_in[c] > 0.  The call
+ *                    does not keep the arrays.
+ *   workspace        >= kvzip_score_context_workspace_size(B, G, max n_in[c])
+ *                    bytes, as for kvzip_score_chunk.
+ *
+ * Other arguments as for kvzip_score_chunk.  n_chunks = 0 is a no-op.  On an
+ * error the chunks before the failing one have been enqueued.
  */
 size_t kvzip_score_context_workspace_size(int B, int G, int max_n_in);
-
-/* Step `step` of the pipeline: pass 1 of chunk `step` (q_next [B][G][n_in_next][d],
- * k_self_next [B][n_in_next][d]; both NULL after the last chunk) and pass 2 of
- * chunk `step - 1` (q_prev [B][G][n_in_prev][d]; NULL at step 0) into `scores`.
- * Running steps 0..n_chunks in order on one stream and workspace equals
- * calling kvzip_score_chunk for each chunk in order, up to fp32 rounding of
- * the normalisers (the two kernels sum the exponentials in different orders).
- * Other arguments as for kvzip_score_chunk.  A chunk whose normalisers do not
- * fit a slot is KVZIP_ERR_INVALID_ARG. */
-kvzip_status kvzip_score_pipeline_step(kvzip_dtype dt, int step, const void* q_next,
-                                       const void* k_self_next, int n_in_next,
-                                       const void* q_prev, int n_in_prev, const void* k_ctx,
-                                       float* scores, int B, int G, int n_c, int d, float scale,
-                                       void* workspace, size_t ws_bytes, void* stream);
-
-/* All n_chunks chunks: steps 0..n_chunks of kvzip_score_pipeline_step.
- * q, k_self and n_in are HOST arrays of n_chunks entries (device pointers to
- * each chunk's queries and self keys, and its row count n_in[c] > 0).  The
- * call does not keep the arrays.  n_chunks = 0 is a no-op. */
 kvzip_status kvzip_score_context(kvzip_dtype dt, int n_chunks, const void* const* q,
                                  const void* const* k_self, const int* n_in, const void* k_ctx,
                                  float* scores, int B, int G, int n_c, int d, float scale,

@@ -1,12 +1,11 @@
-"""Multi-chunk scoring through the C ABI (kvzip_score_context and
-kvzip_score_pipeline_step) against the oracle's score_context.
+"""Multi-chunk scoring through the C ABI (kvzip_score_context) against the
+oracle's score_context.
 
 Every chunk of a context is scored into one running maximum (blog post
-section 4.5).  With bf16 and d = 128 the steps after the first run pass 1 of
-chunk c and pass 2 of chunk c - 1 in one kernel; the result must match the
-oracle to the same 2e-3 relative bound as the per-chunk calls, for ragged
-contexts, ragged last chunks, rows of a tile spanning several query heads,
-more work items than SMs, and the unfused shapes (d = 256, one chunk).
+section 4.5).  The one call must match the oracle to the same 2e-3 relative
+bound as the per-chunk calls and give the same bits as calling
+kvzip_score_chunk chunk by chunk, for ragged contexts, ragged last chunks,
+rows of a tile spanning several query heads, many units, d = 256 and fp32.
 """
 import numpy as np
 import pytest
@@ -31,7 +30,7 @@ def f64(t):
     return t.detach().cpu().to(torch.float64).numpy()
 
 
-def make_context(seed, B, G, n_c, d, n_ins, hi_frac=0.02):
+def make_context(seed, B, G, n_c, d, n_ins, hi_frac=0.02, dtype=torch.bfloat16):
     g = torch.Generator().manual_seed(seed)
     k = torch.randn(B, n_c, d, generator=g)
     k = k * torch.where(torch.rand(B, n_c, 1, generator=g) < hi_frac, 3.0, 1.0)
@@ -41,8 +40,8 @@ def make_context(seed, B, G, n_c, d, n_ins, hi_frac=0.02):
         q = torch.randn(B, G, n_in, d, generator=g)
         ks = torch.randn(B, n_in, d, generator=g)
         ks = ks * torch.where(torch.rand(B, n_in, 1, generator=g) < hi_frac, 3.0, 1.0)
-        chunks.append((q.to(torch.bfloat16), ks.to(torch.bfloat16)))
-    return k.to(torch.bfloat16), chunks
+        chunks.append((q.to(dtype), ks.to(dtype)))
+    return k.to(dtype), chunks
 
 
 def oracle_context(k, chunks):
@@ -57,8 +56,8 @@ CONTEXT_SHAPES = [  # (B, G, n_c, d, n_in per chunk)
     (1, 1, 1, 128, (1, 1)),                    # one key, one row per chunk
     (64, 4, 1536, 128, (272, 272)),            # several items of both passes per CTA
     (300, 1, 64, 128, (8, 8, 8)),              # many short items
-    (2, 2, 500, 256, (150, 150)),              # d = 256: passes run back to back
-    (1, 4, 2048, 128, (16,)),                  # one chunk: nothing to pipeline
+    (2, 2, 500, 256, (150, 150)),              # head dim 256
+    (1, 4, 2048, 128, (16,)),                  # one chunk
 ]
 
 
@@ -74,38 +73,27 @@ def test_score_context_matches_oracle(kz, shape):
     ws = kz.new_context_workspace(B, G, max(n_ins))
     kz.score_context(dch, kd, S, ws)
     assert kz.workspace_status(ws) == kz.OK
-    n_launch = kz.last_launch_count()
-    fused = d == 128 and len(n_ins) > 1
-    # fused: one launch per step (first and last step run a single pass)
-    assert n_launch == (len(n_ins) + 1 if fused else 2 * len(n_ins))
+    assert kz.last_launch_count() == 2 * len(n_ins)   # two passes per chunk
     got = S.cpu().double().numpy()
     assert np.all(np.isfinite(got))
     err = float(np.max(np.abs(got - want) / want))
     assert err <= RTOL, err
 
 
-def test_pipeline_steps_equal_context_call(kz):
-    """Driving the steps by hand gives the same bits as kvzip_score_context, and
-    both agree with chunk-by-chunk kvzip_score_chunk to fp32 rounding."""
-    B, G, n_c, d, n_ins = 5, 4, 3000, 128, (300, 300, 300)
-    k, chunks = make_context(11, B, G, n_c, d, n_ins)
-    kd = k.cuda()
-    dch = [(q.cuda(), ks.cuda()) for q, ks in chunks]
-    S_ctx = torch.zeros(B, n_c, device="cuda")
-    kz.score_context(dch, kd, S_ctx)
-    ws = kz.new_context_workspace(B, G, max(n_ins))
-    S_step = torch.zeros(B, n_c, device="cuda")
-    for step in range(len(dch) + 1):
-        nxt = dch[step] if step < len(dch) else None
-        prev = dch[step - 1] if step > 0 else None
-        kz.score_pipeline_step(step, nxt, prev, kd, S_step, ws)
-    assert kz.workspace_status(ws) == kz.OK
-    assert torch.equal(S_ctx, S_step)
-    S_chunk = torch.zeros(B, n_c, device="cuda")
-    for q, ks in dch:
-        kz.score_chunk(q, kd, ks, S_chunk)
-    rel = ((S_ctx - S_chunk).abs() / S_chunk).max().item()
-    assert rel <= 1e-3, rel
+def test_context_call_equals_chunk_calls(kz):
+    """One kvzip_score_context call gives the same bits as kvzip_score_chunk
+    per chunk in order (bf16 and the fp32 CUDA-core path)."""
+    for dtype in (torch.bfloat16, torch.float32):
+        B, G, n_c, d, n_ins = 5, 4, 3000, 128, (300, 300, 131)
+        k, chunks = make_context(11, B, G, n_c, d, n_ins, dtype=dtype)
+        kd = k.cuda()
+        dch = [(q.cuda(), ks.cuda()) for q, ks in chunks]
+        S_ctx = torch.zeros(B, n_c, device="cuda")
+        kz.score_context(dch, kd, S_ctx)
+        S_chunk = torch.zeros(B, n_c, device="cuda")
+        for q, ks in dch:
+            kz.score_chunk(q, kd, ks, S_chunk)
+        assert torch.equal(S_ctx, S_chunk), dtype
 
 
 def test_context_running_max_over_existing_scores(kz):
@@ -121,22 +109,20 @@ def test_context_running_max_over_existing_scores(kz):
     assert float(np.max(np.abs(got - want) / want)) <= RTOL
 
 
-def test_pipeline_timeout_reported_and_context_survives(kz):
-    """The fused step's bounded waits: with the loaders held back, every CTA
-    gives up after 10 ms, reports KVZIP_ERR_TIMEOUT and writes no scores;
-    afterwards the same steps succeed."""
+def test_context_timeout_reported_and_context_survives(kz):
+    """With the loaders held back, every CTA of every chunk gives up after
+    10 ms, the call reports KVZIP_ERR_TIMEOUT through the status word and no
+    score is written; afterwards the same call succeeds."""
     B, G, n_c, d, n_ins = 4, 4, 4096, 128, (300, 300)
     k, chunks = make_context(14, B, G, n_c, d, n_ins)
     kd = k.cuda()
     dch = [(q.cuda(), ks.cuda()) for q, ks in chunks]
     ws = kz.new_context_workspace(B, G, max(n_ins))
     S = torch.zeros(B, n_c, device="cuda")
-    kz.score_pipeline_step(0, dch[0], None, kd, S, ws)   # chunk 0 normalisers
-    assert kz.workspace_status(ws) == kz.OK
     kz.set_wait_timeout_ns(10_000_000)
     kz.set_test_stall(True)
     try:
-        kz.score_pipeline_step(1, dch[1], dch[0], kd, S, ws)
+        kz.score_context(dch, kd, S, ws)
         status = kz.workspace_status(ws)
     finally:
         kz.set_test_stall(False)
@@ -144,7 +130,6 @@ def test_pipeline_timeout_reported_and_context_survives(kz):
     assert status == kz.ERR_TIMEOUT
     assert torch.count_nonzero(S) == 0
     assert kz.workspace_status(ws) == kz.OK
-    S.zero_()
     kz.score_context(dch, kd, S, ws)
     assert kz.workspace_status(ws) == kz.OK
     want = oracle_context(k, chunks)
@@ -158,7 +143,7 @@ def test_context_rejects_bad_arguments(kz):
     kd = k.cuda()
     dch = [(q.cuda(), ks.cuda()) for q, ks in chunks]
     S = torch.zeros(B, n_c, device="cuda")
-    small = kz.new_context_workspace(B, G, 32)   # slots too small for the 400-row chunk
+    small = kz.new_context_workspace(B, G, 32)   # too small for the 400-row chunk
     assert kz.context_workspace_size(B, G, 400) > small.numel()
     with pytest.raises(kz.KvzipError):
         kz.score_context(dch, kd, S, small)
