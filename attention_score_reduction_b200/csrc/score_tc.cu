@@ -404,14 +404,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               best += a0 + a1;
             } else {
-              float b0 = best, b1 = -INFINITY;
+              // min over rows of lse2 - c*s (packed pairs), i.e. minus the running max
+              const float2 nc2 = make_float2(-c, -c);
+              float w0 = -best, w1 = INFINITY;
 #pragma unroll
               for (int j = 0; j < CH; j += 4) {
                 const float4 L = L4[(ch + j) / 4];   // same address in every lane: broadcast
-                b0 = fmax3(b0, fmaf(v[j + 0], c, -L.x), fmaf(v[j + 1], c, -L.y));
-                b1 = fmax3(b1, fmaf(v[j + 2], c, -L.z), fmaf(v[j + 3], c, -L.w));
+                const float2 x01 = ffma2(make_float2(v[j + 0], v[j + 1]), nc2, make_float2(L.x, L.y));
+                const float2 x23 = ffma2(make_float2(v[j + 2], v[j + 3]), nc2, make_float2(L.z, L.w));
+                w0 = fmin3(w0, x01.x, x01.y);
+                w1 = fmin3(w1, x23.x, x23.y);
               }
-              best = fmaxf(b0, b1);
+              best = -fminf(w0, w1);
             }
           }
           mbar_arrive(&l_empty[st]);

@@ -105,13 +105,15 @@ __global__ void __launch_bounds__(kHistThreads)
   const int64_t n4 = (gridDim.y == 1 || N % 4 == 0) ? N / 4 : 0;
   const uint4* s4 = reinterpret_cast<const uint4*>(s);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  // two independent 16-byte loads in flight per thread
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
-       i += stride) {
-    const uint4 u = __ldcs(s4 + i);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+       i += 2 * stride) {
+    const uint4 u0 = __ldcs(s4 + i);
+    const uint4 u1 = (i + stride < n4) ? __ldcs(s4 + i + stride) : make_uint4(~0u, ~0u, ~0u, ~0u);
+    const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
-      if ((w[e] & PM) == prefix) atomicAdd(&h[(w[e] >> SH) & (NB - 1)], 1u);
+    for (int e = 0; e < 8; ++e)   // all-ones (a NaN pattern) never matches a prefix of a score
+      if (w[e] != ~0u && (w[e] & PM) == prefix) atomicAdd(&h[(w[e] >> SH) & (NB - 1)], 1u);
   }
   for (int64_t i = 4 * n4 + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < N;
        i += stride) {
@@ -230,6 +232,123 @@ __global__ void __launch_bounds__(kSelThreads)
     uint32_t t = 0;
     for (int w = 0; w < kSelThreads / 32; ++w) t += red[w];
     blk_eq[blk] = t;
+  }
+}
+
+// Vector forms of the two passes below for n_c a multiple of 4: each thread
+// reads four consecutive scores with one 16-byte load (two loads in flight)
+// and writes their four mask bytes with one 4-byte store.
+__global__ void __launch_bounds__(kSelThreads)
+    sel_eqcount_v(const float* __restrict__ s, int64_t n_c, int64_t segs, const SelState* st,
+                  uint32_t* blk_eq, int per_head) {
+  const int64_t blk = blockIdx.x;
+  const int64_t h = blk / segs, sg = blk % segs;
+  if (per_head) st += h;
+  if (st->keep_none || st->take_eq == st->n_eq) return;
+  const int64_t j0 = sg * kSelSeg, n4 = (imin64(j0 + kSelSeg, n_c) - j0) / 4;
+  const uint4* b4 = reinterpret_cast<const uint4*>(s + h * n_c + j0);
+  const uint32_t tau = st->tau;
+  uint32_t c = 0;
+  for (int64_t i = threadIdx.x; i < n4; i += 2 * kSelThreads) {
+    const uint4 u0 = __ldcs(b4 + i);
+    const uint4 u1 = (i + kSelThreads < n4) ? __ldcs(b4 + i + kSelThreads) : make_uint4(~0u, ~0u, ~0u, ~0u);
+    c += (u0.x == tau) + (u0.y == tau) + (u0.z == tau) + (u0.w == tau) + (u1.x == tau) +
+         (u1.y == tau) + (u1.z == tau) + (u1.w == tau);
+  }
+  __shared__ uint32_t red[kSelThreads / 32];
+  c = __reduce_add_sync(0xffffffffu, c);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t t = 0;
+    for (int w = 0; w < kSelThreads / 32; ++w) t += red[w];
+    blk_eq[blk] = t;
+  }
+}
+
+__device__ __forceinline__ uint32_t mask4(uint4 u, uint32_t tau, bool eq_keeps) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  uint32_t m = 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    m |= static_cast<uint32_t>(w[e] > tau || (eq_keeps && w[e] == tau)) << (8 * e);
+  return m;
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+    sel_mask_v(const float* __restrict__ s, int64_t n_c, int64_t segs, const SelState* st,
+               const uint32_t* blk_eq_base, uint8_t* keep, uint32_t* blk_cnt, int per_head) {
+  const int64_t blk = blockIdx.x;
+  const int64_t h = blk / segs, sg = blk % segs;
+  if (per_head) st += h;
+  const int64_t j0 = sg * kSelSeg, n4 = (imin64(j0 + kSelSeg, n_c) - j0) / 4;
+  const uint4* b4 = reinterpret_cast<const uint4*>(s + h * n_c + j0);
+  uint32_t* k4 = reinterpret_cast<uint32_t*>(keep + h * n_c + j0);
+  const bool none = st->keep_none != 0;
+  const uint32_t tau = st->tau;
+  const bool rank_ties = !none && st->take_eq != st->n_eq;
+  const unsigned long long take_eq = st->take_eq;
+  __shared__ uint32_t wsum[kSelThreads / 32];
+  __shared__ uint32_t red[kSelThreads / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t kept = 0;
+  if (none) {
+    for (int64_t i = threadIdx.x; i < n4; i += kSelThreads) k4[i] = 0u;
+  } else if (!rank_ties) {   // every score >= tau is kept
+    for (int64_t i = threadIdx.x; i < n4; i += 2 * kSelThreads) {
+      const bool in1 = i + kSelThreads < n4;
+      const uint4 u0 = __ldcs(b4 + i);
+      const uint4 u1 = in1 ? __ldcs(b4 + i + kSelThreads) : make_uint4(0, 0, 0, 0);
+      const uint32_t m0 = mask4(u0, tau, true), m1 = in1 ? mask4(u1, tau, true) : 0u;
+      k4[i] = m0;
+      if (in1) k4[i + kSelThreads] = m1;
+      kept += __popc(m0) + __popc(m1);   // one set bit per kept byte
+    }
+  } else {                   // rank the scores equal to tau in flat order
+    unsigned long long tie_before = blk_eq_base[blk];
+    for (int64_t ib = 0; ib < n4; ib += kSelThreads) {
+      const int64_t i = ib + threadIdx.x;
+      const bool in = i < n4;
+      const uint4 u = in ? __ldcs(b4 + i) : make_uint4(0, 0, 0, 0);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      uint32_t c_eq = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) c_eq += (in && w[e] == tau);
+      uint32_t incl = c_eq;   // inclusive scan over the warp's lanes (flat order)
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+      }
+      if (lane == 31) wsum[warp] = incl;
+      __syncthreads();
+      uint32_t before = 0, total = 0;
+      for (int ww = 0; ww < kSelThreads / 32; ++ww) {
+        before += (ww < warp) ? wsum[ww] : 0;
+        total += wsum[ww];
+      }
+      unsigned long long rank = tie_before + before + incl - c_eq;
+      uint32_t m = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool eq = in && w[e] == tau;
+        const bool k = (in && w[e] > tau) || (eq && rank < take_eq);
+        rank += eq;
+        m |= static_cast<uint32_t>(k) << (8 * e);
+      }
+      if (in) k4[i] = m;
+      kept += __popc(m);
+      tie_before += total;
+      __syncthreads();
+    }
+  }
+  kept = __reduce_add_sync(0xffffffffu, kept);
+  if (lane == 0) red[warp] = kept;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t t = 0;
+    for (int ww = 0; ww < kSelThreads / 32; ++ww) t += red[ww];
+    blk_cnt[blk] = t;
   }
 }
 
@@ -362,7 +481,14 @@ size_t select_ws_bytes(int64_t N, int64_t n_heads) {
   return 256 + align_up(kHistTotal * 4, 256) + 2 * align_up(static_cast<size_t>(nblk) * 4, 256);
 }
 
+// The vector passes need every head's scores on 16 bytes and its mask bytes on 4.
+static bool use_vec(const SelectArgs& a) {
+  return a.n_c % 4 == 0 && reinterpret_cast<uintptr_t>(a.scores) % 16 == 0 &&
+         reinterpret_cast<uintptr_t>(a.keep) % 4 == 0;
+}
+
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launches) {
+  const bool vec = use_vec(a);
   const int64_t segs = segs_per_head(a.n_c);
   const int64_t nblk = a.n_heads * segs;
   SelWs w = carve(a.ws, nblk);
@@ -381,13 +507,21 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launches) {
     sel_pick<1><<<1, kPickThreads, 0, s>>>(w.st, w.hist, a.threshold);
     sel_hist<2><<<grid, kHistThreads, 0, s>>>(a.scores, a.N, w.st, w.hist);
     sel_pick<2><<<1, kPickThreads, 0, s>>>(w.st, w.hist, a.threshold);
-    sel_eqcount<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs, w.st,
-                                                                   w.blk_eq, 0);
+    if (vec)
+      sel_eqcount_v<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs,
+                                                                       w.st, w.blk_eq, 0);
+    else
+      sel_eqcount<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs,
+                                                                     w.st, w.blk_eq, 0);
     sel_scan_blocks<<<1, kPickThreads, 0, s>>>(w.blk_eq, nblk, w.st, 1);
     n += 8;
   }
-  sel_mask<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs, w.st,
-                                                              w.blk_eq, a.keep, w.blk_cnt, 0);
+  if (vec)
+    sel_mask_v<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs, w.st,
+                                                                  w.blk_eq, a.keep, w.blk_cnt, 0);
+  else
+    sel_mask<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs, w.st,
+                                                                w.blk_eq, a.keep, w.blk_cnt, 0);
   sel_offsets<<<1, kPickThreads, 0, s>>>(w.blk_cnt, a.n_heads, segs, a.offsets);
   n += 2;
   if (launches) *launches += n;
@@ -401,6 +535,7 @@ size_t select_per_head_ws_bytes(int64_t n_heads, int64_t n_c) {
 // Uniform head budgets: the same radix selection run for every head at once
 // (grid dimension = head), k_per_head pairs kept in each.
 cudaError_t launch_select_per_head(const SelectArgs& a, cudaStream_t s, int* launches) {
+  const bool vec = use_vec(a);
   const int64_t segs = segs_per_head(a.n_c);
   const int64_t nblk = a.n_heads * segs;
   uint8_t* p = static_cast<uint8_t*>(a.ws);
@@ -428,13 +563,21 @@ cudaError_t launch_select_per_head(const SelectArgs& a, cudaStream_t s, int* lau
     sel_pick<1><<<H, kPickThreads, 0, s>>>(st, hist, nullptr);
     sel_hist<2><<<grid, kHistThreads, 0, s>>>(a.scores, a.n_c, st, hist);
     sel_pick<2><<<H, kPickThreads, 0, s>>>(st, hist, nullptr);
-    sel_eqcount<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs, st,
-                                                                   blk_eq, 1);
+    if (vec)
+      sel_eqcount_v<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs,
+                                                                       st, blk_eq, 1);
+    else
+      sel_eqcount<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs,
+                                                                     st, blk_eq, 1);
     sel_scan_blocks<<<H, kPickThreads, 0, s>>>(blk_eq, segs, st, 1);
     n += 8;
   }
-  sel_mask<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs, st, blk_eq,
-                                                              a.keep, blk_cnt, 1);
+  if (vec)
+    sel_mask_v<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs, st,
+                                                                  blk_eq, a.keep, blk_cnt, 1);
+  else
+    sel_mask<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs, st,
+                                                                blk_eq, a.keep, blk_cnt, 1);
   sel_offsets<<<1, kPickThreads, 0, s>>>(blk_cnt, a.n_heads, segs, a.offsets);
   n += 2;
   if (launches) *launches += n;

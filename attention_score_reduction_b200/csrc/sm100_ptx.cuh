@@ -407,6 +407,11 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   return p;
 }
 
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float y;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+  return y;
+}
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float y;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));

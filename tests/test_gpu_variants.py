@@ -81,3 +81,38 @@ def test_select_per_head(kz, n_heads, n_c, levels, r):
     keep, off = kz.select_per_head(s.cuda(), k_h)
     assert np.array_equal(keep.cpu().numpy(), keep_ref)
     assert np.array_equal(off.cpu().numpy(), off_ref)
+
+
+@pytest.mark.parametrize("n_heads,n_c", [(256, 16384), (7, 1001), (3, 4), (1, 5)])
+def test_head_scores(kz, n_heads, n_c):
+    """Head-level scores max_j S[h][j] (rebuttal, head-level scores): bit-exact,
+    from aligned rows (16-byte loads) and from a view that starts 4 bytes in."""
+    from attention_score_reduction_b200 import synth
+    s = synth.random_scores(n_heads, n_c, seed=n_c + 3)
+    want = oracle.head_scores(s.numpy(), 1, n_heads).reshape(-1).astype(np.float32)
+    got = kz.head_scores(s.cuda()).cpu().numpy()
+    assert np.array_equal(got, want)
+    flat = torch.zeros(n_heads * n_c + 1, device="cuda")
+    flat[1:] = s.reshape(-1).cuda()
+    got2 = kz.head_scores(flat[1:].view(n_heads, n_c)).cpu().numpy()
+    assert np.array_equal(got2, want)
+
+
+def test_token_scores_and_select_from_unaligned_views(kz):
+    """The 16-byte paths are taken only for aligned rows: token scores from a view
+    that starts 4 bytes into its buffer, and a selection mask written at an odd
+    address, go through the scalar kernels and give the same bits."""
+    from attention_score_reduction_b200 import synth
+    n_heads, n_c = 12, 4096
+    s = synth.random_scores(n_heads, n_c, seed=23, levels=5)
+    flat = torch.zeros(n_heads * n_c + 1, device="cuda")
+    flat[1:] = s.reshape(-1).cuda()
+    view = flat[1:].view(n_heads, n_c)
+    assert np.array_equal(kz.token_scores(view).cpu().numpy(),
+                          oracle.token_scores(s.numpy()).astype(np.float32))
+    k = kz.keep_count(0.3, s.numel())
+    keep_ref, off_ref, _ = oracle.select(s.reshape(-1).numpy(), k, n_heads)
+    buf = torch.zeros(n_heads * n_c + 4, dtype=torch.uint8, device="cuda")
+    keep_view = buf[1:1 + n_heads * n_c]            # mask bytes off 4-byte alignment
+    kz.select(s.reshape(-1).cuda(), k, n_heads, keep=keep_view)   # scores must be aligned
+    assert np.array_equal(keep_view.cpu().numpy(), keep_ref)
