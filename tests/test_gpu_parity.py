@@ -235,3 +235,38 @@ def test_head_scores_bit_exact(kz, n_heads, n_c):
     L = 1
     want = oracle.head_scores(s.numpy(), L, n_heads)[0]
     assert np.array_equal(got, want.astype(np.float32))
+
+
+@pytest.mark.parametrize("jump", [70.0, 130.0])
+def test_score_chunk_late_dominant_key(kz, jump):
+    """A context key far down the sequence outscores every earlier key by `jump`
+    in log2 units (all query rows share one direction, the key is a multiple of
+    it), far past the range of the pass-1 polynomial and of fp32 exponentials
+    taken against any earlier maximum.  The online maximum must rescale the
+    row sum exactly.  Scores above 1e-30 match the oracle to 2e-3, the rest
+    are below 1e-30."""
+    B, G, n_in, n_c, d = 2, 2, 40, 2000, 128
+    g = torch.Generator().manual_seed(int(jump))
+    u = torch.randn(d, generator=g)
+    q = (u.repeat(B, G, n_in, 1) + 0.05 * torch.randn(B, G, n_in, d, generator=g)).to(torch.bfloat16)
+    k = torch.randn(B, n_c, d, generator=g)
+    ks = torch.randn(B, n_in, d, generator=g)
+    c = 1.4426950408889634 / np.sqrt(d)
+    beta = jump / (c * float(u @ u))
+    # two keys: at d = 128 (96-key tiles, 48-column chunks, polynomial on the
+    # first 4 of every 16 columns) key 1488 lands on the polynomial, 1500 on MUFU
+    k[:, 1488] = beta * u
+    k[:, 1500] = beta * u
+    k, ks = k.to(torch.bfloat16), ks.to(torch.bfloat16)
+    want = oracle_scores(q, k, ks, torch.zeros(B, n_c))
+    S = torch.zeros(B, n_c, device="cuda")
+    ws = kz.new_score_workspace(B, G, n_in)
+    kz.score_chunk(q.cuda(), k.cuda(), ks.cuda(), S, ws)
+    assert kz.workspace_status(ws) == kz.OK
+    got = S.cpu().double().numpy()
+    assert np.all(np.isfinite(got))
+    assert got[:, [1488, 1500]].min() > 0.49
+    big = want > 1e-30
+    assert float(np.max(np.abs(got[big] - want[big]) / want[big])) <= RTOL
+    if (~big).any():
+        assert float(np.max(np.abs(got[~big]))) <= 1e-30
