@@ -171,3 +171,30 @@ def test_decode_rejects_bad_arguments(kz):
     assert call(q=FAKE + 8) == kz.ERR_INVALID_ARG
     assert call(wsb=16) == kz.ERR_INVALID_ARG
     assert kz.decode_workspace_size(8, 4, 128) > 0
+
+
+def test_score_context_rejects_bad_arguments(kz):
+    """kvzip_score_context validates its host arrays and the workspace before
+    enqueueing anything (no GPU needed for any of these)."""
+    lib = kz.library()
+    vp = ctypes.c_void_p
+    q = (vp * 2)(FAKE, FAKE)
+    ks = (vp * 2)(FAKE, FAKE)
+    n_in = (ctypes.c_int * 2)(16, 16)
+    ws_ok = lib.kvzip_score_context_workspace_size(2, 4, 16)
+    assert ws_ok == lib.kvzip_score_workspace_size(2, 4, 16)
+
+    def call(n, qa=q, ka=ks, na=n_in, ws=ws_ok):
+        return lib.kvzip_score_context(kz.BF16, n, qa, ka, na, FAKE, FAKE, 2, 4, 64, 128, 0.0,
+                                       FAKE, ws, None)
+    assert call(-1) == kz.ERR_INVALID_ARG
+    assert call(0) == kz.OK                                  # nothing to score
+    assert call(2, qa=None) == kz.ERR_INVALID_ARG
+    assert call(2, ka=None) == kz.ERR_INVALID_ARG
+    assert call(2, na=None) == kz.ERR_INVALID_ARG
+    assert call(2, qa=(vp * 2)(FAKE, None)) == kz.ERR_INVALID_ARG
+    assert call(2, na=(ctypes.c_int * 2)(16, 0)) == kz.ERR_INVALID_ARG
+    assert call(2, ws=ws_ok - 1) == kz.ERR_INVALID_ARG       # workspace too small
+    # the largest chunk sets the workspace: 16 and 1000 rows need the 1000-row size
+    big = (ctypes.c_int * 2)(16, 1000)
+    assert call(2, na=big) == kz.ERR_INVALID_ARG
