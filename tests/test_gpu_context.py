@@ -52,9 +52,9 @@ CONTEXT_SHAPES = [  # (B, G, n_c, d, n_in per chunk)
     (2, 4, 300, 128, (100, 100, 37)),          # ragged tails, ragged last chunk
     (3, 2, 1000, 128, (17, 17)),               # a row tile spans several query heads
     (2, 5, 777, 128, (200, 200, 120)),         # G = 5 (Qwen2.5-14B grouping)
-    (1, 4, 2048, 128, (528, 528, 528, 528)),   # tile multiples, three fused steps
+    (1, 4, 2048, 128, (528, 528, 528, 528)),   # tile multiples, four chunks
     (1, 1, 1, 128, (1, 1)),                    # one key, one row per chunk
-    (64, 4, 1536, 128, (272, 272)),            # several items of both passes per CTA
+    (64, 4, 1536, 128, (272, 272)),            # more CTAs than SMs in both passes
     (300, 1, 64, 128, (8, 8, 8)),              # many short items
     (2, 2, 500, 256, (150, 150)),              # head dim 256
     (1, 4, 2048, 128, (16,)),                  # one chunk
