@@ -253,8 +253,9 @@ def test_score_chunk_late_dominant_key(kz, jump):
     ks = torch.randn(B, n_in, d, generator=g)
     c = 1.4426950408889634 / np.sqrt(d)
     beta = jump / (c * float(u @ u))
-    # two keys: at d = 128 (96-key tiles, 48-column chunks, polynomial on the
-    # first 4 of every 16 columns) key 1488 lands on the polynomial, 1500 on MUFU
+    # two keys: the polynomial takes the first 4 of every 16 accumulator columns
+    # (tiles and chunks start on multiples of 16), so key 1488 lands on the
+    # polynomial and key 1500 on MUFU
     k[:, 1488] = beta * u
     k[:, 1500] = beta * u
     k, ks = k.to(torch.bfloat16), ks.to(torch.bfloat16)
