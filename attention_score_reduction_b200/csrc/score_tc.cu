@@ -15,12 +15,14 @@
 //   c * s - lse2[rho]; exp is monotone, so one exp2 per key at the end:
 //   p_j = 2^(max_rho (c s_rho,j - lse2[rho])).
 //
-// One skeleton serves both passes.  The A tile of a CTA never changes, so it
-// lives in tensor memory: each epilogue thread copies its own row there once
-// (tcgen05.st), and every MMA reads A from TMEM and only B from shared memory
-// (tcgen05.mma with A in TMEM).  That halves the shared-memory operand traffic
-// per MMA, which otherwise limits a 128 x N x 16 MMA with both operands in
-// shared memory to about half the tensor core's rate on B200.
+// One skeleton serves both passes.  The A tiles of a CTA never change.  Where
+// TMEM has room (pass 1, and d = 256) they live in tensor memory: each epilogue
+// thread copies its own row there once, before any MMA (tcgen05.st), and every
+// MMA reads A from TMEM and only B from shared memory.  Pass 2 at d = 128 uses
+// wider B tiles instead (N = 128, a quarter fewer tiles, each with its own
+// barrier waits and commits; measured 62 against 66 ms per 128K chunk): the four
+// 128-column accumulators fill TMEM, so its A tiles are loaded by TMA into
+// shared memory and the MMAs read both operands there (tile sizes in TcCfg).
 //   warp 0      : TMA producer, a STAGES-deep ring of B tiles (+ pass-2 lse2 tiles)
 //   warps 1, 2  : one MMA-issuing thread each, for A tile 0 and A tile 1 (warp 1
 //                 also allocates TMEM).  tcgen05.mma issue stalls until the
@@ -49,17 +51,29 @@
 
 namespace kvzip {
 
-template <int D>
+// Tile configuration per head dimension and pass.
+template <int D, bool PASS2>
 struct TcCfg;
 template <>
-struct TcCfg<128> {
+struct TcCfg<128, false> {           // pass 1 at d = 128
   static constexpr int BN = 96;      // rows per B tile (N of the MMA)
   static constexpr int STAGES = 6;   // B ring depth
+  static constexpr bool A_SMEM = false;  // A tiles in TMEM (tcgen05.st once per CTA)
+  static constexpr int CH = 48;          // accumulator columns per TMEM load
 };
 template <>
-struct TcCfg<256> {
+struct TcCfg<128, true> {            // pass 2 at d = 128
+  static constexpr int BN = 128;
+  static constexpr int STAGES = 4;
+  static constexpr bool A_SMEM = true;   // A tiles in shared memory (TMA): TMEM holds 4 x 128
+  static constexpr int CH = 32;          // accumulator columns
+};
+template <bool PASS2>
+struct TcCfg<256, PASS2> {
   static constexpr int BN = 64;
   static constexpr int STAGES = 5;
+  static constexpr bool A_SMEM = false;
+  static constexpr int CH = 32;
 };
 
 constexpr int kEpiThreads = 512;     // four 128-thread epilogue groups
@@ -74,15 +88,20 @@ constexpr int kATiles = 2;           // A tiles per CTA
 #endif
 constexpr int kPolyPairs = KVZIP_POLY_PAIRS;
 
-template <int D>
+template <int D, bool PASS2>
 struct TcLayout {
-  static constexpr int BN = TcCfg<D>::BN;
-  static constexpr int STAGES = TcCfg<D>::STAGES;
+  using Cfg = TcCfg<D, PASS2>;
+  static constexpr int BN = Cfg::BN;
+  static constexpr int STAGES = Cfg::STAGES;
   static constexpr int KB = D / 64;                      // 128-byte K blocks per row
+  static constexpr bool A_SMEM = Cfg::A_SMEM;
   static constexpr int B_KB_BYTES = BN * 128;
   static constexpr int B_BYTES = KB * B_KB_BYTES;
   static constexpr int L_BYTES = BN * 4;                 // pass 2: lse2 of one B tile
-  static constexpr int OFF_B = 0;
+  static constexpr int A_KB_BYTES = kBM * 128;
+  static constexpr int A_TILE_BYTES = KB * A_KB_BYTES;   // one A tile in shared memory
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + (A_SMEM ? kATiles * A_TILE_BYTES : 0);
   static constexpr int OFF_L = OFF_B + STAGES * B_BYTES;
   static constexpr int OFF_BAR = OFF_L + STAGES * L_BYTES;
   // barriers: a_full, b_full[S], b_empty[S], s_full[2][2], s_empty[2][2], mma_done, l_empty[S]
@@ -90,15 +109,18 @@ struct TcLayout {
   static constexpr int OFF_XCHG = OFF_BAR + 8 * N_BARS;  // parity merge, float2 per row
   static constexpr int OFF_MISC = OFF_XCHG + kATiles * kBM * 8;  // tmem base, abort flag
   static constexpr int BYTES = OFF_MISC + 16;
-  static constexpr int CH = BN / 2;                      // accumulator columns per TMEM load
+  static constexpr int CH = Cfg::CH;                     // accumulator columns per TMEM load
   static constexpr int SMEM_ALLOC = BYTES + 1024;        // slack for 1024-B alignment
-  static constexpr int A_COLS = D / 2;                   // TMEM columns of one A tile
+  static constexpr int A_COLS = A_SMEM ? 0 : D / 2;      // TMEM columns of one A tile
   static constexpr int ACC0 = kATiles * A_COLS;          // first accumulator column
   static constexpr int TMEM_COLS = 512;
   static_assert(ACC0 + kATiles * 2 * BN <= TMEM_COLS, "TMEM over-committed");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "invalid MMA N");
   static_assert(SMEM_ALLOC <= 232448, "exceeds 227 KB of shared memory");
-  static_assert((B_KB_BYTES % 1024) == 0, "swizzle atoms must stay 1024-B aligned");
+  static_assert((B_KB_BYTES % 1024) == 0 && (A_KB_BYTES % 1024) == 0,
+                "swizzle atoms must stay 1024-B aligned");
+  static_assert(BN % CH == 0, "tile not a multiple of the TMEM load");
+  static_assert(!A_SMEM || BN == kBM, "A tiles are loaded with the B maps' box height");
 };
 
 struct TcParams {
@@ -117,8 +139,10 @@ struct TcParams {
 template <int D, bool PASS2, bool SUM = false>
 __global__ void __launch_bounds__(kThreads, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap bmap0,
-                    const __grid_constant__ CUtensorMap bmap1, const TcParams p) {
-  using Lay = TcLayout<D>;
+                    const __grid_constant__ CUtensorMap bmap1,
+                    const __grid_constant__ CUtensorMap amap,   // A rows, box kBM (A_SMEM only)
+                    const TcParams p) {
+  using Lay = TcLayout<D, PASS2>;
   constexpr int BN = Lay::BN;
   constexpr int STAGES = Lay::STAGES;
   constexpr int KB = Lay::KB;
@@ -157,7 +181,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   if (threadIdx.x == 0) {
-    mbar_init(a_full, nA * kBM);   // every thread of every active group stores its A row
+    // A in TMEM: every thread of every active group stores its row; A in shared
+    // memory: one TMA transaction
+    mbar_init(a_full, Lay::A_SMEM ? 1 : nA * kBM);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&b_full[s], 1);
       mbar_init(&b_empty[s], nA);   // one commit per active MMA issuer
@@ -188,6 +214,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&bmap0);
       if (!PASS2) tma_prefetch_desc(&bmap1);
       const bool stall = p.test_stall != 0;
+      if (Lay::A_SMEM && !stall) {   // the CTA's A tiles (rows past the operand read as zeros)
+        tma_prefetch_desc(&amap);
+        mbar_arrive_expect_tx(a_full, nA * Lay::A_TILE_BYTES);
+        for (int t = 0; t < nA; ++t)
+          for (int kb = 0; kb < KB; ++kb)
+            tma_load_3d(smem + Lay::OFF_A + t * Lay::A_TILE_BYTES + kb * Lay::A_KB_BYTES, &amap,
+                        a_full, kb * 64, a_row0 + t * kBM, b);
+      }
       int issued = 0;
 #pragma unroll 1
       for (int it = 0; !stall && it < n_b; ++it) {
@@ -215,6 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int last = s + ((issued - 1 - s) / STAGES) * STAGES;
         wait_drain(&b_full[s], (last / STAGES) & 1, p.status);
       }
+      if (Lay::A_SMEM && !stall) wait_drain(a_full, 0, p.status);
     }
     __syncwarp();
   } else if (warp <= kATiles) {
@@ -224,6 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
       const uint32_t b_base = smem_u32(smem + Lay::OFF_B);
       const uint32_t a_tmem = tmem_base + t * Lay::A_COLS;
+      const uint32_t a_sbase = smem_u32(smem + Lay::OFF_A + t * Lay::A_TILE_BYTES);
       bool ok = wait_one(a_full, 0, ctl);
       tc_fence_after();
 #pragma unroll 1
@@ -237,10 +273,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kb = 0; kb < KB; ++kb) {
           const uint64_t bd = sdesc_sw128(b_base + s * Lay::B_BYTES + kb * Lay::B_KB_BYTES);
+          if (Lay::A_SMEM) {
+            const uint64_t ad = sdesc_sw128(a_sbase + kb * Lay::A_KB_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)   // K = 16 per MMA: 8 TMEM columns of A, 32 B of B
-            umma_bf16_ts(d_tmem, a_tmem + (kb * 4 + kk) * 8, bd + 2 * kk, idesc,
-                         (kb | kk) != 0);
+            for (int kk = 0; kk < 4; ++kk)   // K = 16 per MMA: 32 B of each row
+              umma_bf16_ss(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)   // K = 16 per MMA: 8 TMEM columns of A, 32 B of B
+              umma_bf16_ts(d_tmem, a_tmem + (kb * 4 + kk) * 8, bd + 2 * kk, idesc,
+                           (kb | kk) != 0);
+          }
         }
         umma_commit(&s_full[t * 2 + buf]);
         umma_commit(&b_empty[s]);
@@ -263,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = p.c;
     float2* xchg = reinterpret_cast<float2*>(smem + Lay::OFF_XCHG) + t * kBM + lrow;
     if (t < nA) {
-      if (par == 0) {
+      if (!Lay::A_SMEM && par == 0) {
         // ---- this thread's A row into its TMEM lane (zeros past the operand's rows)
         const uint4* src = reinterpret_cast<const uint4*>(
             p.a_ptr + (static_cast<size_t>(b) * a_extent + arow) * D);
@@ -456,17 +499,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D>
 static cudaError_t launch_tc(const ScoreArgs& a, cudaStream_t s, int* launches) {
-  using Lay = TcLayout<D>;
+  using L1 = TcLayout<D, false>;
+  using L2 = TcLayout<D, true>;
   // The shared-memory limit is a per-device function attribute; set it each call.
   cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<D, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       Lay::SMEM_ALLOC);
+                                       L1::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(score_tc_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           Lay::SMEM_ALLOC);
+                           L2::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(score_tc_kernel<D, true, true>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM_ALLOC);
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, L2::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
   TcParams p;
   p.a_ptr = static_cast<const uint16_t*>(a.q);
@@ -482,29 +526,33 @@ static cudaError_t launch_tc(const ScoreArgs& a, cudaStream_t s, int* launches) 
   p.timeout_ns = a.timeout_ns;
   p.test_stall = a.test_stall;
 
+  // Maps of box height BN (per pass).  With A in shared memory (BN = kBM) a map
+  // of the A operand serves the A tiles; with A in TMEM its rows are copied from
+  // global memory by the epilogue threads and the A map is not read.
   if (a.passes & 1) {
-    // B operands only: A rows go straight from global memory into TMEM.
     CUtensorMap kmap, smap;
-    if (!make_map(&kmap, a.k_ctx, a.B, a.n_c, D, Lay::BN) ||
-        !make_map(&smap, a.k_self, a.B, a.n_in, D, Lay::BN))
+    if (!make_map(&kmap, a.k_ctx, a.B, a.n_c, D, L1::BN) ||
+        !make_map(&smap, a.k_self, a.B, a.n_in, D, L1::BN))
       return cudaErrorInvalidValue;
     dim3 g1((a.R + kATiles * kBM - 1) / (kATiles * kBM), a.B);
-    score_tc_kernel<D, false><<<g1, kThreads, Lay::SMEM_ALLOC, s>>>(kmap, smap, p);
+    score_tc_kernel<D, false><<<g1, kThreads, L1::SMEM_ALLOC, s>>>(kmap, smap, kmap, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (launches) *launches += 1;
   }
   if (!(a.passes & 2)) return cudaSuccess;
 
-  // pass 2: A = context key tiles (TMEM), B = query row tiles (box BN rows)
-  CUtensorMap qmapB;
-  if (!make_map(&qmapB, a.q, a.B, a.R, D, Lay::BN)) return cudaErrorInvalidValue;
+  // pass 2: A = context key tiles, B = query row tiles
+  CUtensorMap kmap2, qmap2;
+  if (!make_map(&kmap2, a.k_ctx, a.B, a.n_c, D, L2::BN) ||
+      !make_map(&qmap2, a.q, a.B, a.R, D, L2::BN))
+    return cudaErrorInvalidValue;
   p.a_ptr = static_cast<const uint16_t*>(a.k_ctx);
   dim3 g2((a.n_c + kATiles * kBM - 1) / (kATiles * kBM), a.B);
   if (a.sum_aggregation)
-    score_tc_kernel<D, true, true><<<g2, kThreads, Lay::SMEM_ALLOC, s>>>(qmapB, qmapB, p);
+    score_tc_kernel<D, true, true><<<g2, kThreads, L2::SMEM_ALLOC, s>>>(qmap2, qmap2, kmap2, p);
   else
-    score_tc_kernel<D, true><<<g2, kThreads, Lay::SMEM_ALLOC, s>>>(qmapB, qmapB, p);
+    score_tc_kernel<D, true><<<g2, kThreads, L2::SMEM_ALLOC, s>>>(qmap2, qmap2, kmap2, p);
   e = cudaGetLastError();
   if (e == cudaSuccess && launches) *launches += 1;
   return e;
