@@ -23,7 +23,8 @@
 // barrier waits and commits; measured 62 against 66 ms per 128K chunk): the four
 // 128-column accumulators fill TMEM, so its A tiles are loaded by TMA into
 // shared memory and the MMAs read both operands there (tile sizes in TcCfg).
-//   warp 0      : TMA producer, a STAGES-deep ring of B tiles (+ pass-2 lse2 tiles)
+//   warp 0      : TMA producer: the A tiles when they live in shared memory, then
+//                 a STAGES-deep ring of B tiles (+ pass-2 lse2 tiles)
 //   warps 1, 2  : one MMA-issuing thread each, for A tile 0 and A tile 1 (warp 1
 //                 also allocates TMEM).  tcgen05.mma issue stalls until the
 //                 previous MMA is nearly done, so one thread's barrier waits and
@@ -31,12 +32,13 @@
 //                 instead of 64 cycles per 128x128x16 MMA); with two issuers one
 //                 feeds the pipe while the other waits.
 //   warps 3..18 : four 128-thread epilogue groups, one per (A tile, accumulator
-//                 buffer); the even group of each A tile first copies the A
-//                 rows into TMEM.  A group drains its BN-column accumulator in
-//                 two TMEM loads, so the tile's B tiles alternate between two
-//                 groups (four epilogue warps per scheduler: the epilogue math
-//                 is latency-bound with two).
-// TMEM map (512 columns): [0, 2*D/2) A tiles, then (tile, buffer) accumulators.
+//                 buffer); with A in TMEM the even group of each A tile first
+//                 copies the A rows there.  A group drains its BN-column
+//                 accumulator in CH-column TMEM loads, so the tile's B tiles
+//                 alternate between two groups (four epilogue warps per
+//                 scheduler: the epilogue math is latency-bound with two).
+// TMEM map (512 columns): the A tiles when they live there (D/2 columns each),
+// then the (tile, buffer) accumulators.
 // Every wait is bounded; on timeout the CTA records KVZIP_ERR_TIMEOUT in the
 // status word, drains its in-flight copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
