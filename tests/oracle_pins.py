@@ -385,23 +385,83 @@ def pin_sum_aggregation(o):
     assert abs(cs.sum() + self_mass - G * n_in) < 1e-12
 
 
-def pin_token_and_uniform_budgets(o):
-    """Token-level scores are the per-position max over heads; uniform budgets
-    keep exactly k_h per head, each head's kept set being its own top k_h
-    (checked by the defining property), and an all-heads position mask
-    expands to identical per-head masks."""
+def pin_uniform_budgets(o):
+    """Uniform budgets keep exactly k_h per head, each head's kept set being its
+    own top k_h with ties taken lowest position first (the defining property,
+    checked head by head)."""
     r = _rng(71)
     S = (np.floor(r.random((4, 30)) * 6) / 6).astype(np.float32)
-    tok = o.token_scores(S)
-    assert np.array_equal(tok, S.max(axis=0).astype(np.float64))
     keep, off = o.select_per_head(S.reshape(-1), 9, 4)
     assert np.array_equal(off, [0, 9, 18, 27, 36])
     for h in range(4):
-        _check_selection(S[h], 9, 1, keep.reshape(4, 30)[h], np.array([0, 9]), S[h][keep.reshape(4, 30)[h] == 1].min())
-    kp = np.zeros(30, np.uint8)
-    kp[[1, 5, 7]] = 1
-    ke, offe = o.expand_keep(kp, 4)
-    assert np.array_equal(ke.reshape(4, 30), np.tile(kp, (4, 1))) and offe[-1] == 12
+        kh = keep.reshape(4, 30)[h]
+        _check_selection(S[h], 9, 1, kh, np.array([0, 9]), S[h][kh == 1].min())
+
+
+def _planted_scores(L, H, n_c, cells, seed):
+    """Background scores in [0, 0.5) with hand-placed larger values at the given
+    (l, h, j) cells.  Pure-Python lists, no array reductions."""
+    r = _rng(seed)
+    S = [[[0.5 * float(r.random()) for _ in range(n_c)] for _ in range(H)] for _ in range(L)]
+    for (l, h, j), val in cells.items():
+        S[l][h][j] = val
+    return S
+
+
+def pin_head_scores(o):
+    """Head-level scores (rebuttal, answer on the head-level scores used for the
+    DuoAttention comparison: the maximum over the sequence axis of the
+    L x H x n_c score tensor).  L = 3, H = 2, n_c = 5 with one planted maximum
+    per head at a hand-chosen position; the expected value of head (l, h) is the
+    value planted there, written out by hand, and a pure-Python triple loop over
+    (l, h, j) agrees."""
+    L, H, n_c = 3, 2, 5
+    planted = {(0, 0, 4): 0.91, (0, 1, 0): 0.62, (1, 0, 2): 0.97,
+               (1, 1, 1): 0.55, (2, 0, 0): 0.88, (2, 1, 3): 0.73}
+    S = _planted_scores(L, H, n_c, planted, seed=72)
+    want = [[0.91, 0.62], [0.97, 0.55], [0.88, 0.73]]
+    loop = [[max(S[l][h][j] for j in range(n_c)) for h in range(H)] for l in range(L)]
+    assert loop == want
+    got = o.head_scores(np.array(S), L, H)
+    assert np.shape(got) == (L, H), np.shape(got)
+    for l in range(L):
+        for h in range(H):
+            assert float(got[l][h]) == want[l][h], (l, h, got[l][h])
+
+
+def pin_token_scores(o):
+    """Token-level scores (blog post section 4.3.3: one score per position, the
+    maximum over all layers and heads).  Each position's maximum is planted in
+    a different (layer, head), including heads other than the first and layers
+    other than the first, so a maximum over layers only or over heads only
+    misses some of them.  Input as [L, H, n_c] and as [L*H, n_c]."""
+    L, H, n_c = 3, 2, 6
+    planted = {(2, 1, 0): 0.93, (0, 1, 1): 0.81, (1, 0, 2): 0.77,
+               (0, 0, 3): 0.99, (2, 0, 4): 0.66, (1, 1, 5): 0.58}
+    S = _planted_scores(L, H, n_c, planted, seed=73)
+    want = [0.93, 0.81, 0.77, 0.99, 0.66, 0.58]
+    loop = [max(S[l][h][j] for l in range(L) for h in range(H)) for j in range(n_c)]
+    assert loop == want
+    for arr in (np.array(S), np.array(S).reshape(L * H, n_c)):
+        got = o.token_scores(arr)
+        assert np.shape(got) == (n_c,), np.shape(got)
+        assert [float(x) for x in got] == want
+
+
+def pin_expand_keep(o):
+    """A position mask shared by all heads (token-level eviction, blog post
+    section 4.3.3) becomes one identical row per head, and head h's packed rows
+    start after h full copies of the kept positions.  Checked by loops against
+    hand-written expectations."""
+    n_heads, n_c = 4, 7
+    kp = [0, 1, 0, 0, 1, 1, 0]                       # kept positions 1, 4, 5
+    keep, off = o.expand_keep(np.array(kp, np.uint8), n_heads)
+    keep = np.asarray(keep).reshape(-1)
+    assert keep.size == n_heads * n_c
+    for h in range(n_heads):
+        for j in range(n_c):
+            assert int(keep[h * n_c + j]) == kp[j], (h, j)
+    assert [int(x) for x in off] == [0, 3, 6, 9, 12]
 
 
 SCORING_PINS = [pin_row_sums_and_range, pin_uniform_queries, pin_logistic, pin_dominant_key,
@@ -409,5 +469,6 @@ SCORING_PINS = [pin_row_sums_and_range, pin_uniform_queries, pin_logistic, pin_d
 SELECT_PINS = [pin_keep_count, pin_select_properties, pin_select_bruteforce]
 COMPACT_PINS = [pin_compact, pin_kv_size_table]
 DECODE_PINS = [pin_decode_closed_forms, pin_decode_matches_dense_over_kept]
-VARIANT_PINS = [pin_sum_aggregation, pin_token_and_uniform_budgets]
+VARIANT_PINS = [pin_sum_aggregation, pin_uniform_budgets, pin_head_scores, pin_token_scores,
+                pin_expand_keep]
 ALL_PINS = SCORING_PINS + SELECT_PINS + COMPACT_PINS + DECODE_PINS + VARIANT_PINS

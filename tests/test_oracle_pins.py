@@ -178,11 +178,53 @@ def _mut_per_head_tie_high(m):
     m.select_per_head = sph
 
 
+def _mut_head_scores_wrong_axis(m):
+    # maximum over the heads of a layer instead of over the positions of a head
+    m.head_scores = lambda S, L, H: np.asarray(S, np.float64).reshape(L, H, -1).max(axis=1)
+
+
+def _mut_head_scores_heads_major(m):
+    # units read as head-major (h * L + l) instead of layer-major (l * H + h)
+    m.head_scores = lambda S, L, H: np.asarray(S, np.float64).reshape(H, L, -1).max(axis=2).T
+
+
+def _mut_token_scores_layers_only(m):
+    # maximum over the leading axis only: layers, not layers and heads
+    m.token_scores = lambda S: np.asarray(S, np.float64).max(axis=0)
+
+
+def _mut_token_scores_first_head(m):
+    # maximum over the layers of the first head of each layer only
+    def tok(S):
+        S = np.asarray(S, np.float64)
+        n_c = S.shape[-1]
+        return S.reshape(-1, n_c)[::2].max(axis=0)
+    m.token_scores = tok
+
+
+def _mut_expand_repeat(m):
+    # each position repeated n_heads times instead of the whole mask per head
+    def expand(keep_pos, n_heads):
+        kp = np.asarray(keep_pos).astype(np.uint8).reshape(-1)
+        return np.repeat(kp, n_heads), np.arange(n_heads + 1, dtype=np.int64) * int(kp.sum())
+    m.expand_keep = expand
+
+
+def _mut_expand_offsets_by_n_c(m):
+    # head h's rows start at h * n_c (the dense layout) instead of h * kept
+    def expand(keep_pos, n_heads):
+        kp = np.asarray(keep_pos).astype(np.uint8).reshape(-1)
+        return np.tile(kp, n_heads), np.arange(n_heads + 1, dtype=np.int64) * kp.size
+    m.expand_keep = expand
+
+
 MUTANTS = [_mut_drop_diagonal, _mut_anticausal, _mut_row_order, _mut_no_self_in_normaliser,
            _mut_no_scale, _mut_mean, _mut_sum_over_chunks, _mut_transposed_keys,
            _mut_floor_count, _mut_tie_high_index, _mut_uniform_head_budget,
            _mut_positions_descending, _mut_decode_no_scale, _mut_decode_wrong_head,
-           _mut_sum_without_self, _mut_per_head_tie_high]
+           _mut_sum_without_self, _mut_per_head_tie_high, _mut_head_scores_wrong_axis,
+           _mut_head_scores_heads_major, _mut_token_scores_layers_only,
+           _mut_token_scores_first_head, _mut_expand_repeat, _mut_expand_offsets_by_n_c]
 
 
 @pytest.mark.parametrize("mutate", MUTANTS, ids=lambda f: f.__name__)
