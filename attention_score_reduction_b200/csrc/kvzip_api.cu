@@ -25,6 +25,8 @@ kvzip_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KVZIP_OK : KVZ
 
 }  // namespace
 
+void kvzip::note_launches(int launches) { g_last_launches.store(launches); }
+
 extern "C" {
 
 const char* kvzip_status_string(kvzip_status s) {
@@ -46,6 +48,15 @@ void kvzip_set_test_stall(int on) { g_test_stall.store(on ? 1 : 0); }
 
 /* Number of kernel launches the most recent successful call enqueued (testing aid). */
 int kvzip_last_launch_count(void) { return g_last_launches.load(); }
+
+kvzip_status kvzip_score_lse_layout(int G, int n_in, size_t* offset_bytes, int64_t* row_stride) {
+  if (G <= 0 || n_in <= 0 || !offset_bytes || !row_stride) return KVZIP_ERR_INVALID_ARG;
+  const int64_t R = static_cast<int64_t>(G) * n_in;
+  if (R > INT_MAX - kvzip::kRowPad) return KVZIP_ERR_UNSUPPORTED;
+  *offset_bytes = kvzip::kScoreWsHeader;
+  *row_stride = row_pad(R);
+  return KVZIP_OK;
+}
 
 size_t kvzip_score_workspace_size(int B, int G, int n_in) {
   if (B < 0 || G < 0 || n_in < 0) return 0;
@@ -190,13 +201,10 @@ kvzip_status kvzip_select(const float* scores, int64_t N, int64_t k, int64_t n_h
     return KVZIP_ERR_INVALID_ARG;
   if (ws_bytes < kvzip_select_workspace_size(N, n_heads)) return KVZIP_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (N == 0) {  // no scores: every head keeps nothing
-    cudaError_t e = cudaMemsetAsync(offsets, 0, sizeof(int64_t) * (n_heads + 1), s);
-    if (e == cudaSuccess && threshold) {
-      const float inf = INFINITY;
-      e = cudaMemcpyAsync(threshold, &inf, sizeof(float), cudaMemcpyHostToDevice, s);
-      if (e == cudaSuccess) e = cudaStreamSynchronize(s);  // `inf` lives on this stack frame
-    }
+  if (N == 0) {  // no scores: every head keeps nothing (one enqueued kernel, no sync)
+    int launches = 0;
+    const cudaError_t e = kvzip::launch_select_empty(offsets, n_heads, threshold, s, &launches);
+    if (e == cudaSuccess) g_last_launches.store(launches);
     return from_cuda(e);
   }
   kvzip::SelectArgs a;

@@ -14,8 +14,9 @@ constexpr uint32_t kStatusTimeout = 1u;
 constexpr size_t kScoreWsHeader = 256;
 
 // Query rows of one unit are padded to a multiple of this many in the
-// log-sum-exp buffer (a multiple of the pass-1 CTA's 256 rows and of every
-// pass-2 query tile height: 96 and 64).
+// log-sum-exp buffer.  Pass 2 reads whole query tiles of it (128 rows at
+// d = 128, 64 at d = 256) and pass 1 pads in steps of its 256-row CTAs; the
+// scorer asserts at compile time that this divides by both.
 constexpr int kRowPad = 768;
 
 struct ScoreArgs {
@@ -53,6 +54,9 @@ size_t select_ws_bytes(int64_t N, int64_t n_heads);
 size_t select_per_head_ws_bytes(int64_t n_heads, int64_t n_c);
 cudaError_t launch_select_per_head(const SelectArgs& a, cudaStream_t s, int* launches);
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launches);
+// N = 0: zero offsets, threshold +inf, on the stream.
+cudaError_t launch_select_empty(int64_t* offsets, int64_t n_heads, float* threshold,
+                                cudaStream_t s, int* launches);
 
 struct CompactArgs {
   const void* k;
@@ -98,5 +102,8 @@ int decode_splits(int64_t n_heads);
 size_t decode_ml_bytes(int64_t n_heads, int G);
 size_t decode_ws_bytes(int64_t n_heads, int G, int d);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, int* launches);
+
+// Records the launch count of an accepted call (read by kvzip_last_launch_count).
+void note_launches(int launches);
 
 }  // namespace kvzip

@@ -123,6 +123,10 @@ struct TcLayout {
                 "swizzle atoms must stay 1024-B aligned");
   static_assert(BN % CH == 0, "tile not a multiple of the TMEM load");
   static_assert(!A_SMEM || BN == kBM, "A tiles are loaded with the B maps' box height");
+  // Pass 2 copies whole BN-row tiles of lse2 up to the padded row count, and
+  // pass 1 pads it in steps of its CTA height: both must divide the pad.
+  static_assert(kRowPad % BN == 0 && kRowPad % (kATiles * kBM) == 0,
+                "row pad of the log-sum-exp buffer must divide by every tile height");
 };
 
 struct TcParams {

@@ -52,7 +52,7 @@ struct SelWs {
 };
 
 // Radix rounds of 13 + 10 + 9 bits: bins, shift of the digit, bits fixed before
-// the round, histogram offset.  Scores in (0, 1] share few exponents, so the
+// the round, histogram offset.  Scores in [0, 1] share few exponents, so the
 // first round takes 5 mantissa bits along with sign and exponent to spread
 // them over enough shared-memory bins to keep atomic contention low.
 __host__ __device__ constexpr int hist_bins(int p) { return p == 0 ? 8192 : (p == 1 ? 1024 : 512); }
@@ -528,6 +528,20 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launches) {
   return cudaGetLastError();
 }
 
+// No scores at all: every head keeps nothing and the threshold is +inf.  One
+// block writes the outputs so that the call stays asynchronous.
+__global__ void sel_empty(int64_t* offsets, int64_t n_heads, float* threshold) {
+  for (int64_t i = threadIdx.x; i <= n_heads; i += blockDim.x) offsets[i] = 0;
+  if (threadIdx.x == 0 && threshold) *threshold = INFINITY;
+}
+
+cudaError_t launch_select_empty(int64_t* offsets, int64_t n_heads, float* threshold,
+                                cudaStream_t s, int* launches) {
+  sel_empty<<<1, 256, 0, s>>>(offsets, n_heads, threshold);
+  if (launches) *launches += 1;
+  return cudaGetLastError();
+}
+
 size_t select_per_head_ws_bytes(int64_t n_heads, int64_t n_c) {
   return per_head_ws_bytes(n_heads, n_c);
 }
@@ -611,19 +625,27 @@ void* g_scratch_ptr[kMaxDevices] = {};
 std::mutex g_scratch_mu;
 
 // Device address of g_select_scratch on the current device.  In host code the
-// array's name is only a host-side stand-in, so the address is looked up once
-// per device (with that device current) and cached.
-cudaError_t static_scratch(void** out) {
+// array's name is only a host-side stand-in, so the address is looked up with
+// that device current.  Outside stream capture it is looked up on every call
+// (cheap), so a context torn down and re-created (cudaDeviceReset) gets its new
+// address; while `stream` is capturing, the address cached by an earlier call
+// on this device is used, because the lookup may have to load the module.
+cudaError_t static_scratch(cudaStream_t stream, void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(stream, &cap);
+  if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_select_scratch);
     if (e != cudaSuccess) return e;
     g_scratch_ptr[dev] = p;
+  } else if (!g_scratch_ptr[dev]) {
+    return cudaErrorStreamCaptureUnsupported;
   }
   *out = g_scratch_ptr[dev];
   return cudaSuccess;
@@ -644,7 +666,8 @@ extern "C" kvzip_status kvzip_select_noalloc(const float* scores, int64_t N, int
   // Larger problems need more scratch than the static array holds.
   if (kvzip::select_ws_bytes(N, n_heads) > kvzip::kSelectStaticBytes) return KVZIP_ERR_UNSUPPORTED;
   void* ws = nullptr;
-  if (kvzip::static_scratch(&ws) != cudaSuccess) return KVZIP_ERR_CUDA;
+  if (kvzip::static_scratch(static_cast<cudaStream_t>(stream), &ws) != cudaSuccess)
+    return KVZIP_ERR_CUDA;
   kvzip::SelectArgs a;
   a.scores = scores;
   a.N = N;
@@ -658,5 +681,7 @@ extern "C" kvzip_status kvzip_select_noalloc(const float* scores, int64_t N, int
   a.ws_bytes = kvzip::kSelectStaticBytes;
   int launches = 0;
   const cudaError_t e = kvzip::launch_select(a, static_cast<cudaStream_t>(stream), &launches);
-  return e == cudaSuccess ? KVZIP_OK : KVZIP_ERR_CUDA;
+  if (e != cudaSuccess) return KVZIP_ERR_CUDA;
+  kvzip::note_launches(launches);
+  return KVZIP_OK;
 }

@@ -42,11 +42,13 @@ def _load() -> ctypes.CDLL:
         "kvzip_score_context": (i32, [i32, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, vp,
                                       sz, vp]),
         "kvzip_workspace_status": (i32, [vp, vp]),
+        "kvzip_score_lse_layout": (i32, [i32, i32, ctypes.POINTER(sz), ctypes.POINTER(i64)]),
         "kvzip_set_wait_timeout_ns": (None, [u64]),
         "kvzip_set_test_stall": (None, [i32]),
         "kvzip_keep_count": (i64, [f64, i64]),
         "kvzip_select_workspace_size": (sz, [i64, i64]),
         "kvzip_select": (i32, [vp, i64, i64, i64, vp, vp, vp, vp, sz, vp]),
+        "kvzip_select_noalloc": (i32, [vp, i64, i64, i64, vp, vp, vp, vp]),
         "kvzip_compact_workspace_size": (sz, [i64, i32]),
         "kvzip_compact": (i32, [vp, vp, vp, vp, i64, i32, i32, vp, vp, vp, vp, sz, vp]),
         "kvzip_head_scores": (i32, [vp, i64, i64, vp, vp]),
@@ -211,12 +213,21 @@ def set_test_stall(on: bool):
     _lib.kvzip_set_test_stall(1 if on else 0)
 
 
+def lse_layout(G: int, n_in: int) -> tuple[int, int]:
+    """(byte offset, row stride) of the row normalisers inside a scoring workspace."""
+    off = ctypes.c_size_t(0)
+    stride = ctypes.c_int64(0)
+    _check(_lib.kvzip_score_lse_layout(G, n_in, ctypes.byref(off), ctypes.byref(stride)),
+           "kvzip_score_lse_layout")
+    return int(off.value), int(stride.value)
+
+
 def read_lse(workspace: torch.Tensor, B: int, G: int, n_in: int) -> torch.Tensor:
     """Natural-log row normalisers the last pass-1 launch left in the workspace,
-    [B][G*n_in] (a view into the workspace's padded buffer, converted)."""
+    [B][G*n_in] (the library stores base-2 values; converted here)."""
     R = G * n_in
-    R_pad = (R + 767) // 768 * 768
-    lse2 = workspace[256:256 + B * R_pad * 4].view(torch.float32).view(B, R_pad)[:, :R]
+    off, stride = lse_layout(G, n_in)
+    lse2 = workspace[off:off + B * stride * 4].view(torch.float32).view(B, stride)[:, :R]
     return lse2 * 0.6931471805599453
 
 

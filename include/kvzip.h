@@ -74,6 +74,10 @@ size_t kvzip_score_workspace_size(int B, int G, int n_in);
  *             scores[b][j] = max(scores[b][j], max_rho P[b][rho][j]) where
  *             P[b][rho][:] = softmax over (n_c context logits, i+1 self logits)
  *             of scale * q . k.  Zero it before the first chunk; 4-byte aligned.
+ *             Results lie in [0, 1]: the method's probabilities are > 0, but
+ *             the fp32 exponential flushes values below 2^-126 (the smallest
+ *             normal float) to 0, so a key whose best probability is below
+ *             that scores 0 (and is evicted first).
  *   scale   <= 0 or NaN selects 1/sqrt(d).
  *   d       128 or 256.
  *   workspace / ws_bytes: >= kvzip_score_workspace_size(B, G, n_in) bytes,
@@ -128,6 +132,18 @@ kvzip_status kvzip_score_context(kvzip_dtype dt, int n_chunks, const void* const
                                  const void* const* k_self, const int* n_in, const void* k_ctx,
                                  float* scores, int B, int G, int n_c, int d, float scale,
                                  void* workspace, size_t ws_bytes, void* stream);
+
+/* Where kvzip_score_lse (and the first half of kvzip_score_chunk) leaves the
+ * row normalisers in the workspace, for callers that read them: the float32 of
+ * unit b, query row rho = g*n_in + i, sits at byte
+ *     *offset_bytes + 4 * (b * *row_stride + rho)
+ * and holds the base-2 log-sum-exp of the row's scaled logits,
+ *     log2( sum over its n_c context and i+1 visible self keys of
+ *           2^(scale * log2(e) * q . k) ),
+ * i.e. the natural-log normaliser times log2(e).  Rows rho >= G*n_in up to
+ * the stride are padding.  Valid after the launch completes; the next scoring
+ * call on the same workspace overwrites it.  Host-only, no CUDA call. */
+kvzip_status kvzip_score_lse_layout(int G, int n_in, size_t* offset_bytes, int64_t* row_stride);
 
 /* Synchronise `stream`, then report (and clear) the status word the scoring
  * kernels leave in `workspace`: KVZIP_OK, or KVZIP_ERR_TIMEOUT when a kernel

@@ -198,3 +198,21 @@ def test_score_context_rejects_bad_arguments(kz):
     # the largest chunk sets the workspace: 16 and 1000 rows need the 1000-row size
     big = (ctypes.c_int * 2)(16, 1000)
     assert call(2, na=big) == kz.ERR_INVALID_ARG
+
+
+def test_score_lse_layout(kz):
+    """The row normalisers sit after the 256-byte status header, one row stride
+    per unit, the stride being the unit's G * n_in rows rounded up to the pad;
+    the workspace size covers exactly that."""
+    for G, n_in in [(4, 2064), (5, 2064), (2, 1040), (1, 1), (4, 129)]:
+        off, stride = kz.lse_layout(G, n_in)
+        assert off == 256
+        assert stride >= G * n_in and stride % 128 == 0 and stride - G * n_in < 768
+        B = 7
+        assert kz.score_workspace_size(B, G, n_in) == off + B * stride * 4
+    lib = kz.library()
+    o, s = ctypes.c_size_t(0), ctypes.c_int64(0)
+    assert lib.kvzip_score_lse_layout(0, 10, ctypes.byref(o), ctypes.byref(s)) == kz.ERR_INVALID_ARG
+    assert lib.kvzip_score_lse_layout(4, 10, None, ctypes.byref(s)) == kz.ERR_INVALID_ARG
+    assert lib.kvzip_score_lse_layout(1 << 20, 1 << 20, ctypes.byref(o),
+                                      ctypes.byref(s)) == kz.ERR_UNSUPPORTED

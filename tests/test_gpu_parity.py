@@ -171,6 +171,25 @@ def test_select_config_shape_scores(kz):
     assert int(off[-1]) == k == 1258292
 
 
+def test_select_no_scores(kz):
+    """N = 0: every head keeps nothing and the threshold is +inf, written by one
+    enqueued kernel (the call does not synchronise)."""
+    n_heads = 5
+    s = torch.empty(0, dtype=torch.float32, device="cuda")
+    keep = torch.empty(0, dtype=torch.uint8, device="cuda")
+    off = torch.full((n_heads + 1,), -7, dtype=torch.int64, device="cuda")
+    thr = torch.zeros(1, dtype=torch.float32, device="cuda")
+    nws = kz.select_workspace_size(0, n_heads)
+    ws = torch.empty(nws, dtype=torch.uint8, device="cuda")
+    st = kz.library().kvzip_select(None, 0, 0, n_heads, None, off.data_ptr(), thr.data_ptr(),
+                                   ws.data_ptr(), nws, torch.cuda.current_stream().cuda_stream)
+    assert st == kz.OK and kz.last_launch_count() == 1
+    torch.cuda.synchronize()
+    assert off.tolist() == [0] * (n_heads + 1)
+    assert float(thr.item()) == float("inf")
+    del keep, s
+
+
 # ------------------------------------------------------------------ compaction
 
 @pytest.mark.parametrize("d", [128, 256])

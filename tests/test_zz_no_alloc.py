@@ -44,18 +44,24 @@ def test_noalloc_select_matches_workspace_select_twice(lib):
     L, kz = lib
     from attention_score_reduction_b200 import synth
     cases = [(256, 16384, 0, 0.3),    # LLaMA3.1-8B 16K score shape
-             (24, 9000, 4, 0.5)]      # tie-heavy, ragged segments
+             (24, 9000, 4, 0.5),      # tie-heavy, ragged segments
+             (384, 174080, 0, 0.3),   # Gemma3-12B 170K score shape (48 x 8 heads)
+             (40, 5000, 0, 0.0)]      # k = 0: the histogram rounds are skipped
     for n_heads, n_c, levels, r in cases:
         s = synth.random_scores(n_heads, n_c, seed=n_c, levels=levels).reshape(-1).cuda()
         k = kz.keep_count(r, s.numel())
         keep_ref, off_ref, thr_ref = kz.select(s, k, n_heads)
+        launches_ref = kz.last_launch_count()
         st, keep, off, thr = _noalloc(L, s, k, n_heads)
         torch.cuda.synchronize()
         assert st == kz.OK
+        assert kz.last_launch_count() == launches_ref
         assert torch.equal(keep, keep_ref)
         assert torch.equal(off, off_ref)
         assert torch.equal(thr, thr_ref)
         assert int(off[-1]) == k
+        if k == 0:
+            assert not bool(keep.any()) and float(thr.item()) == float("inf")
 
 
 def test_noalloc_select_rejects_oversize(lib):
