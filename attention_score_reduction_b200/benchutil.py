@@ -115,6 +115,12 @@ def load_peaks(path: str) -> dict:
                 "source": "fallback"}
 
 
+def clock_peak_tflops(sms: int, sm_mhz: float) -> float:
+    """Dense bf16 tensor peak at a given SM clock: each SM's tcgen05 pipe does one
+    128 x 128 x 16 MMA in 64 cycles (8192 flop per clock)."""
+    return sms * 8192.0 * sm_mhz * 1e6 / 1e12
+
+
 def score_flops(B: int, G: int, n_in: int, n_c: int, d: int) -> dict:
     """Algorithmic QK^T flops of the two scoring passes for one chunk of B units.
 

@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libkvzip.so")
-SOURCES = ["kvzip_api.cu", "score_tc.cu", "score_simt.cu", "select.cu", "compact.cu", "heads.cu", "decode.cu"]
+SOURCES = ["kvzip_api.cu", "score_tc.cu", "score_simt.cu", "select.cu", "select_fused.cu", "compact.cu", "heads.cu", "decode.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

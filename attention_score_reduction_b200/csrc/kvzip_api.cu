@@ -186,7 +186,7 @@ int64_t kvzip_keep_count(double r, int64_t N) {
 
 size_t kvzip_select_workspace_size(int64_t N, int64_t n_heads) {
   if (N < 0 || n_heads <= 0) return 0;
-  return kvzip::select_ws_bytes(N, n_heads);
+  return kvzip::select_fused_ws_bytes(N, n_heads);
 }
 
 kvzip_status kvzip_select(const float* scores, int64_t N, int64_t k, int64_t n_heads,
@@ -219,7 +219,99 @@ kvzip_status kvzip_select(const float* scores, int64_t N, int64_t k, int64_t n_h
   a.ws = workspace;
   a.ws_bytes = ws_bytes;
   int launches = 0;
-  cudaError_t e = kvzip::launch_select(a, s, &launches);
+  cudaError_t e = kvzip::launch_select_fused(a, g_timeout_ns.load(), s, &launches);
+  if (e == cudaSuccess) g_last_launches.store(launches);
+  return from_cuda(e);
+}
+
+int kvzip_select_shard_bins(int round) { return kvzip::shard_bins(round); }
+
+size_t kvzip_select_shard_workspace_size(int64_t N_local, int64_t n_heads_local) {
+  if (N_local < 0 || n_heads_local <= 0) return 0;
+  return kvzip::select_multipass_ws_bytes(N_local, n_heads_local);
+}
+
+static bool shard_args_ok(const float* scores, int64_t N_local, const void* ws, size_t ws_bytes) {
+  return N_local > 0 && N_local < (int64_t{1} << 31) && scores && aligned(scores, 16) && ws &&
+         aligned(ws, 256) && ws_bytes >= kvzip::select_multipass_ws_bytes(1, 1);
+}
+
+kvzip_status kvzip_select_shard_begin(int64_t k, void* workspace, size_t ws_bytes, void* stream) {
+  if (k < 0 || !workspace || !aligned(workspace, 256) ||
+      ws_bytes < kvzip::select_multipass_ws_bytes(1, 1))
+    return KVZIP_ERR_INVALID_ARG;
+  int launches = 0;
+  const cudaError_t e =
+      kvzip::launch_shard_begin(workspace, k, static_cast<cudaStream_t>(stream), &launches);
+  if (e == cudaSuccess) g_last_launches.store(launches);
+  return from_cuda(e);
+}
+
+kvzip_status kvzip_select_shard_hist(const float* scores, int64_t N_local, int round,
+                                     int64_t* hist, void* workspace, size_t ws_bytes,
+                                     void* stream) {
+  if (!shard_args_ok(scores, N_local, workspace, ws_bytes) || round < 0 || round > 2 || !hist ||
+      !aligned(hist, 8))
+    return KVZIP_ERR_INVALID_ARG;
+  int launches = 0;
+  const cudaError_t e = kvzip::launch_shard_hist(scores, N_local, round,
+                                                 reinterpret_cast<long long*>(hist), workspace,
+                                                 static_cast<cudaStream_t>(stream), &launches);
+  if (e == cudaSuccess) g_last_launches.store(launches);
+  return from_cuda(e);
+}
+
+kvzip_status kvzip_select_shard_pick(const int64_t* hist, int round, float* threshold,
+                                     void* workspace, size_t ws_bytes, void* stream) {
+  if (round < 0 || round > 2 || !hist || !aligned(hist, 8) || !workspace ||
+      !aligned(workspace, 256) || ws_bytes < kvzip::select_multipass_ws_bytes(1, 1) ||
+      (threshold && !aligned(threshold, 4)))
+    return KVZIP_ERR_INVALID_ARG;
+  int launches = 0;
+  const cudaError_t e = kvzip::launch_shard_pick(reinterpret_cast<const long long*>(hist), round,
+                                                 threshold, workspace,
+                                                 static_cast<cudaStream_t>(stream), &launches);
+  if (e == cudaSuccess) g_last_launches.store(launches);
+  return from_cuda(e);
+}
+
+kvzip_status kvzip_select_shard_ties(const float* scores, int64_t N_local, int64_t* n_ties,
+                                     void* workspace, size_t ws_bytes, void* stream) {
+  if (!shard_args_ok(scores, N_local, workspace, ws_bytes) || !n_ties || !aligned(n_ties, 8))
+    return KVZIP_ERR_INVALID_ARG;
+  int launches = 0;
+  const cudaError_t e = kvzip::launch_shard_ties(scores, N_local,
+                                                 reinterpret_cast<long long*>(n_ties), workspace,
+                                                 static_cast<cudaStream_t>(stream), &launches);
+  if (e == cudaSuccess) g_last_launches.store(launches);
+  return from_cuda(e);
+}
+
+kvzip_status kvzip_select_shard_mask(const float* scores, int64_t N_local, int64_t n_heads_local,
+                                     const int64_t* tie_counts, int rank, uint8_t* keep,
+                                     int64_t* offsets, void* workspace, size_t ws_bytes,
+                                     void* stream) {
+  if (!shard_args_ok(scores, N_local, workspace, ws_bytes) || n_heads_local <= 0 ||
+      n_heads_local > (int64_t{1} << 24) || N_local % n_heads_local != 0 || rank < 0 ||
+      !tie_counts || !aligned(tie_counts, 8) || !keep || !offsets || !aligned(offsets, 8))
+    return KVZIP_ERR_INVALID_ARG;
+  if (ws_bytes < kvzip::select_multipass_ws_bytes(N_local, n_heads_local))
+    return KVZIP_ERR_INVALID_ARG;
+  kvzip::SelectArgs a;
+  a.scores = scores;
+  a.N = N_local;
+  a.k = 0;
+  a.n_heads = n_heads_local;
+  a.n_c = N_local / n_heads_local;
+  a.keep = keep;
+  a.offsets = offsets;
+  a.threshold = nullptr;
+  a.ws = workspace;
+  a.ws_bytes = ws_bytes;
+  int launches = 0;
+  const cudaError_t e = kvzip::launch_shard_mask(a, reinterpret_cast<const long long*>(tie_counts),
+                                                 rank, static_cast<cudaStream_t>(stream),
+                                                 &launches);
   if (e == cudaSuccess) g_last_launches.store(launches);
   return from_cuda(e);
 }

@@ -49,11 +49,28 @@ struct SelectArgs {
   void* ws;
   size_t ws_bytes;
 };
-size_t select_ws_bytes(int64_t N, int64_t n_heads);
+// One cooperative launch, two reads of the scores (kvzip_select).
+size_t select_fused_ws_bytes(int64_t N, int64_t n_heads);
+cudaError_t launch_select_fused(const SelectArgs& a, uint64_t timeout_ns, cudaStream_t s,
+                                int* launches);
+// Multi-launch radix select with a small workspace (kvzip_select_noalloc and the
+// sharded selection).
+size_t select_multipass_ws_bytes(int64_t N, int64_t n_heads);
+// Sharded selection (heads split across ranks; histograms summed by the caller).
+int shard_bins(int round);
+cudaError_t launch_shard_begin(void* ws, int64_t k, cudaStream_t s, int* launches);
+cudaError_t launch_shard_hist(const float* scores, int64_t N, int round, long long* hist,
+                              void* ws, cudaStream_t s, int* launches);
+cudaError_t launch_shard_pick(const long long* hist, int round, float* threshold, void* ws,
+                              cudaStream_t s, int* launches);
+cudaError_t launch_shard_ties(const float* scores, int64_t N, long long* n_ties, void* ws,
+                              cudaStream_t s, int* launches);
+cudaError_t launch_shard_mask(const SelectArgs& a, const long long* tie_counts, int rank,
+                              cudaStream_t s, int* launches);
 // Uniform head budgets: SelectArgs.k is the budget of every head.
 size_t select_per_head_ws_bytes(int64_t n_heads, int64_t n_c);
 cudaError_t launch_select_per_head(const SelectArgs& a, cudaStream_t s, int* launches);
-cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launches);
+cudaError_t launch_select_multipass(const SelectArgs& a, cudaStream_t s, int* launches);
 // N = 0: zero offsets, threshold +inf, on the stream.
 cudaError_t launch_select_empty(int64_t* offsets, int64_t n_heads, float* threshold,
                                 cudaStream_t s, int* launches);

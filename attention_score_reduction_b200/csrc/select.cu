@@ -87,22 +87,16 @@ __global__ void sel_init(SelState* st, uint32_t* hist, unsigned long long k, flo
   }
 }
 
-// blockIdx.y selects the problem: elements [y * N, (y + 1) * N).
+// This block's share of one radix round's histogram into shared memory: the
+// digit of every score whose higher bits equal `prefix`.
 template <int PASS>
-__global__ void __launch_bounds__(kHistThreads)
-    sel_hist(const float* __restrict__ s, int64_t N, const SelState* st, uint32_t* hist) {
+__device__ __forceinline__ void hist_count(const float* __restrict__ s, int64_t N, uint32_t prefix,
+                                           bool vec, uint32_t* h) {
   constexpr int NB = hist_bins(PASS);
   constexpr int SH = hist_shift(PASS);
   constexpr uint32_t PM = hist_mask(PASS);
-  __shared__ uint32_t h[NB];
-  s += static_cast<size_t>(blockIdx.y) * N;
-  st += blockIdx.y;
-  hist += static_cast<size_t>(blockIdx.y) * kHistTotal;
-  for (int i = threadIdx.x; i < NB; i += blockDim.x) h[i] = 0;
-  __syncthreads();
-  const uint32_t prefix = st->prefix;
   // vector loads need 16-byte aligned problems (N a multiple of 4)
-  const int64_t n4 = (gridDim.y == 1 || N % 4 == 0) ? N / 4 : 0;
+  const int64_t n4 = vec ? N / 4 : 0;
   const uint4* s4 = reinterpret_cast<const uint4*>(s);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   // two independent 16-byte loads in flight per thread
@@ -120,6 +114,20 @@ __global__ void __launch_bounds__(kHistThreads)
     const uint32_t w = __float_as_uint(s[i]);
     if ((w & PM) == prefix) atomicAdd(&h[(w >> SH) & (NB - 1)], 1u);
   }
+}
+
+// blockIdx.y selects the problem: elements [y * N, (y + 1) * N).
+template <int PASS>
+__global__ void __launch_bounds__(kHistThreads)
+    sel_hist(const float* __restrict__ s, int64_t N, const SelState* st, uint32_t* hist) {
+  constexpr int NB = hist_bins(PASS);
+  __shared__ uint32_t h[NB];
+  s += static_cast<size_t>(blockIdx.y) * N;
+  st += blockIdx.y;
+  hist += static_cast<size_t>(blockIdx.y) * kHistTotal;
+  for (int i = threadIdx.x; i < NB; i += blockDim.x) h[i] = 0;
+  __syncthreads();
+  hist_count<PASS>(s, N, st->prefix, gridDim.y == 1 || N % 4 == 0, h);
   __syncthreads();
   for (int i = threadIdx.x; i < NB; i += blockDim.x)
     if (h[i]) atomicAdd(&hist[hist_off(PASS) + i], h[i]);
@@ -150,26 +158,23 @@ __device__ unsigned long long block_incl_scan(unsigned long long v, unsigned lon
   return v + add;
 }
 
-// Find the bin (counting from the top) that holds the k_rem-th largest element.
-template <int PASS>
-__global__ void __launch_bounds__(kPickThreads)
-    sel_pick(SelState* st, const uint32_t* hist, float* threshold) {
+// Find the bin (counting from the top) of histogram h (NB bins of round PASS)
+// that holds the k_rem-th largest element, and narrow the state to it.
+template <int PASS, typename CountT>
+__device__ void pick_impl(SelState* st, const CountT* h, float* threshold) {
   constexpr int NB = hist_bins(PASS);
   constexpr int PER = (NB + kPickThreads - 1) / kPickThreads;  // 8, 1 or 1 bins per thread
   __shared__ unsigned long long sm[32];
   __shared__ int found_bin;
   __shared__ unsigned long long found_above;
-  st += blockIdx.x;                     // one block per selection problem
-  hist += static_cast<size_t>(blockIdx.x) * kHistTotal;
   if (st->keep_none) return;
-  const uint32_t* h = hist + hist_off(PASS);
   // thread t owns bins NB-1-PER*t ... NB-PER*(t+1) (descending)
   unsigned long long mine = 0;
-  uint32_t cnt[PER];
+  unsigned long long cnt[PER];
 #pragma unroll
   for (int j = 0; j < PER; ++j) {
     const int bin = NB - 1 - (PER * static_cast<int>(threadIdx.x) + j);
-    cnt[j] = bin >= 0 ? h[bin] : 0u;
+    cnt[j] = bin >= 0 ? static_cast<unsigned long long>(h[bin]) : 0ull;
     mine += cnt[j];
   }
   const unsigned long long incl = block_incl_scan(mine, sm);
@@ -197,11 +202,19 @@ __global__ void __launch_bounds__(kPickThreads)
     st->k_rem = k_rem - found_above;
     if (PASS == 2) {
       st->tau = st->prefix;
-      st->n_eq = h[bin];
+      st->n_eq = static_cast<unsigned long long>(h[bin]);
       st->take_eq = st->k_rem;
       if (threshold) *threshold = __uint_as_float(st->prefix);
     }
   }
+}
+
+template <int PASS>
+__global__ void __launch_bounds__(kPickThreads)
+    sel_pick(SelState* st, const uint32_t* hist, float* threshold) {
+  // one block per selection problem
+  pick_impl<PASS>(st + blockIdx.x, hist + static_cast<size_t>(blockIdx.x) * kHistTotal +
+                                        hist_off(PASS), threshold);
 }
 
 __device__ __forceinline__ uint32_t warp_excl_prefix(bool flag, uint32_t* total) {
@@ -475,7 +488,7 @@ size_t per_head_ws_bytes(int64_t n_heads, int64_t n_c) {
          2 * align_up(static_cast<size_t>(nblk) * 4, 256);
 }
 
-size_t select_ws_bytes(int64_t N, int64_t n_heads) {
+size_t select_multipass_ws_bytes(int64_t N, int64_t n_heads) {
   const int64_t n_c = n_heads > 0 ? N / n_heads : 0;
   const int64_t nblk = n_heads * segs_per_head(n_c);
   return 256 + align_up(kHistTotal * 4, 256) + 2 * align_up(static_cast<size_t>(nblk) * 4, 256);
@@ -487,7 +500,7 @@ static bool use_vec(const SelectArgs& a) {
          reinterpret_cast<uintptr_t>(a.keep) % 4 == 0;
 }
 
-cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launches) {
+cudaError_t launch_select_multipass(const SelectArgs& a, cudaStream_t s, int* launches) {
   const bool vec = use_vec(a);
   const int64_t segs = segs_per_head(a.n_c);
   const int64_t nblk = a.n_heads * segs;
@@ -598,6 +611,146 @@ cudaError_t launch_select_per_head(const SelectArgs& a, cudaStream_t s, int* lau
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Sharded selection: one context's heads split across ranks (one process per
+// GPU).  Each rank holds a contiguous run of heads, in rank order, so the flat
+// order of the whole context is rank order, then local order.  The radix
+// rounds need the histogram of all ranks: each rank counts its own scores into
+// 64-bit bins, the caller sums the bins over ranks (an all-reduce) and every
+// rank picks the same bin from the sum.  After the last round every rank knows
+// tau and how many scores equal to tau are kept; the caller gathers each
+// rank's count of scores equal to tau, and a rank keeps its ties whose global
+// flat-order rank (ties on earlier ranks, then its own in flat order) is below
+// that number.
+
+namespace {
+
+template <int PASS>
+__global__ void __launch_bounds__(kHistThreads)
+    shard_hist(const float* __restrict__ s, int64_t N, const SelState* st,
+               unsigned long long* out) {
+  constexpr int NB = hist_bins(PASS);
+  __shared__ uint32_t h[NB];
+  for (int i = threadIdx.x; i < NB; i += blockDim.x) h[i] = 0;
+  __syncthreads();
+  if (!st->keep_none) hist_count<PASS>(s, N, st->prefix, true, h);
+  __syncthreads();
+  for (int i = threadIdx.x; i < NB; i += blockDim.x)
+    if (h[i]) atomicAdd(out + i, static_cast<unsigned long long>(h[i]));
+}
+
+template <int PASS>
+__global__ void __launch_bounds__(kPickThreads)
+    shard_pick(SelState* st, const long long* hist, float* threshold) {
+  pick_impl<PASS>(st, hist, threshold);
+}
+
+// Scores equal to tau on this rank.
+__global__ void __launch_bounds__(kSelThreads)
+    shard_ties(const float* __restrict__ s, int64_t N, const SelState* st,
+               unsigned long long* n_ties) {
+  if (st->keep_none) return;
+  const uint32_t tau = st->tau;
+  uint32_t c = 0;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < N;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    c += (__float_as_uint(s[i]) == tau);
+  c = __reduce_add_sync(0xffffffffu, c);
+  if ((threadIdx.x & 31) == 0 && c) atomicAdd(n_ties, static_cast<unsigned long long>(c));
+}
+
+// Turn the global tie quota into this rank's: ties on earlier ranks come first.
+__global__ void shard_localize(SelState* st, const long long* tie_counts, int rank) {
+  if (threadIdx.x != 0 || st->keep_none) return;
+  unsigned long long before = 0;
+  for (int r = 0; r < rank; ++r) before += static_cast<unsigned long long>(tie_counts[r]);
+  const unsigned long long mine = static_cast<unsigned long long>(tie_counts[rank]);
+  const unsigned long long quota = st->take_eq;
+  const unsigned long long left = quota > before ? quota - before : 0ull;
+  st->n_eq = mine;
+  st->take_eq = left < mine ? left : mine;
+}
+
+int hist_grid(int64_t N) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t want = (N / 4 + kHistThreads - 1) / kHistThreads;
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, 4LL * sms)));
+}
+
+}  // namespace
+
+int shard_bins(int round) { return (round >= 0 && round <= 2) ? hist_bins(round) : 0; }
+
+cudaError_t launch_shard_begin(void* ws, int64_t k, cudaStream_t s, int* launches) {
+  SelWs w = carve(ws, 0);
+  sel_init<<<1, 1024, 0, s>>>(w.st, w.hist, static_cast<unsigned long long>(k), nullptr);
+  if (launches) *launches += 1;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_shard_hist(const float* scores, int64_t N, int round, long long* hist,
+                              void* ws, cudaStream_t s, int* launches) {
+  SelWs w = carve(ws, 0);
+  cudaError_t e = cudaMemsetAsync(hist, 0, sizeof(long long) * hist_bins(round), s);
+  if (e != cudaSuccess) return e;
+  const int grid = hist_grid(N);
+  auto* out = reinterpret_cast<unsigned long long*>(hist);
+  if (round == 0) shard_hist<0><<<grid, kHistThreads, 0, s>>>(scores, N, w.st, out);
+  if (round == 1) shard_hist<1><<<grid, kHistThreads, 0, s>>>(scores, N, w.st, out);
+  if (round == 2) shard_hist<2><<<grid, kHistThreads, 0, s>>>(scores, N, w.st, out);
+  if (launches) *launches += 1;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_shard_pick(const long long* hist, int round, float* threshold, void* ws,
+                              cudaStream_t s, int* launches) {
+  SelWs w = carve(ws, 0);
+  if (round == 0) shard_pick<0><<<1, kPickThreads, 0, s>>>(w.st, hist, threshold);
+  if (round == 1) shard_pick<1><<<1, kPickThreads, 0, s>>>(w.st, hist, threshold);
+  if (round == 2) shard_pick<2><<<1, kPickThreads, 0, s>>>(w.st, hist, threshold);
+  if (launches) *launches += 1;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_shard_ties(const float* scores, int64_t N, long long* n_ties, void* ws,
+                              cudaStream_t s, int* launches) {
+  SelWs w = carve(ws, 0);
+  cudaError_t e = cudaMemsetAsync(n_ties, 0, sizeof(long long), s);
+  if (e != cudaSuccess) return e;
+  const int grid = hist_grid(N);
+  shard_ties<<<grid, kSelThreads, 0, s>>>(scores, N, w.st,
+                                          reinterpret_cast<unsigned long long*>(n_ties));
+  if (launches) *launches += 1;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_shard_mask(const SelectArgs& a, const long long* tie_counts, int rank,
+                              cudaStream_t s, int* launches) {
+  const bool vec = use_vec(a);
+  const int64_t segs = segs_per_head(a.n_c);
+  const int64_t nblk = a.n_heads * segs;
+  SelWs w = carve(a.ws, nblk);
+  shard_localize<<<1, 32, 0, s>>>(w.st, tie_counts, rank);
+  if (vec)
+    sel_eqcount_v<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs,
+                                                                     w.st, w.blk_eq, 0);
+  else
+    sel_eqcount<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs, w.st,
+                                                                   w.blk_eq, 0);
+  sel_scan_blocks<<<1, kPickThreads, 0, s>>>(w.blk_eq, nblk, w.st, 1);
+  if (vec)
+    sel_mask_v<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs, w.st,
+                                                                  w.blk_eq, a.keep, w.blk_cnt, 0);
+  else
+    sel_mask<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs, w.st,
+                                                                w.blk_eq, a.keep, w.blk_cnt, 0);
+  sel_offsets<<<1, kPickThreads, 0, s>>>(w.blk_cnt, a.n_heads, segs, a.offsets);
+  if (launches) *launches += 5;
+  return cudaGetLastError();
+}
+
 }  // namespace kvzip
 
 // ---------------------------------------------------------------------------
@@ -664,7 +817,8 @@ extern "C" kvzip_status kvzip_select_noalloc(const float* scores, int64_t N, int
       (threshold && (reinterpret_cast<uintptr_t>(threshold) & 3)))
     return KVZIP_ERR_INVALID_ARG;
   // Larger problems need more scratch than the static array holds.
-  if (kvzip::select_ws_bytes(N, n_heads) > kvzip::kSelectStaticBytes) return KVZIP_ERR_UNSUPPORTED;
+  if (kvzip::select_multipass_ws_bytes(N, n_heads) > kvzip::kSelectStaticBytes)
+    return KVZIP_ERR_UNSUPPORTED;
   void* ws = nullptr;
   if (kvzip::static_scratch(static_cast<cudaStream_t>(stream), &ws) != cudaSuccess)
     return KVZIP_ERR_CUDA;
@@ -680,7 +834,8 @@ extern "C" kvzip_status kvzip_select_noalloc(const float* scores, int64_t N, int
   a.ws = ws;
   a.ws_bytes = kvzip::kSelectStaticBytes;
   int launches = 0;
-  const cudaError_t e = kvzip::launch_select(a, static_cast<cudaStream_t>(stream), &launches);
+  const cudaError_t e =
+      kvzip::launch_select_multipass(a, static_cast<cudaStream_t>(stream), &launches);
   if (e != cudaSuccess) return KVZIP_ERR_CUDA;
   kvzip::note_launches(launches);
   return KVZIP_OK;

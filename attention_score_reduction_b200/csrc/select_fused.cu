@@ -1,0 +1,507 @@
+// Global top-k selection in one cooperative launch, reading the scores twice.
+//
+// Same result as the multi-launch radix selection in select.cu (the k largest
+// of all L x H x n_c scores, equal scores taken lowest flat index first; scime.ai
+// summary "Approach" and "Measured effects" on non-uniform head budgets;
+// rebuttal: S has shape L x H x n_c), with fewer passes over HBM:
+//
+//   A  every block histograms the top 13 bits of the scores in its contiguous
+//      range (read 1); grid barrier.
+//   B  every block finds, from the merged histogram, the bin b1 that holds the
+//      k-th largest score (the same answer in every block).
+//   C  every block reads its range again (read 2) and writes the final mask
+//      byte of every score outside bin b1 (kept iff its bin is above b1).  The
+//      flat indices of the scores inside bin b1 (the candidates) are appended,
+//      in flat order, to the block's own segment of a candidate buffer, and
+//      their next 10 bits are histogrammed; grid barrier.
+//   D  bin b2 of round 2, then a histogram of the last 9 bits over the
+//      candidates that match b1 b2 (gathered by index); grid barrier.
+//   E  bin b3 gives the threshold tau exactly.  If fewer scores equal to tau
+//      are kept than exist, every block counts its candidates equal to tau and,
+//      after a barrier, sums the counts of the blocks before it: the flat-order
+//      rank of its first tie.
+//   F  every block sets the mask of its kept candidates; grid barrier.
+//   G  block 0 turns the per-head kept counts into offsets and writes tau.
+//
+// Per-head kept counts are accumulated on the way (C and F) by run-length
+// counting per thread: a thread's scores are visited in increasing flat order,
+// so its head only changes at head boundaries.
+//
+// The blocks wait on one another, so the kernel is launched cooperatively (all
+// blocks resident).  Every grid-barrier wait is bounded: on timeout the block
+// records KVZIP_ERR_TIMEOUT in the workspace status word, raises an abort flag
+// that releases the other blocks, and the kernel returns with an incomplete
+// mask.
+#include <cooperative_groups.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "kvzip.h"
+#include "kvzip_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace kvzip {
+namespace {
+
+constexpr int kThr = 512;                // threads per block
+constexpr int kTile = kThr * 4;          // scores per block tile (4 per thread, 16-byte loads)
+constexpr int kMaxBlocks = 1024;
+constexpr int kBins1 = 8192, kBins2 = 1024, kBins3 = 512;
+constexpr int kShift1 = 19, kShift2 = 9;  // digit of round 1: bits 31..19, round 2: 18..9, round 3: 8..0
+
+// Workspace layout (bytes).  [kOffSync, zero_end) is zeroed by the host before
+// every launch; the rest is written before it is read.
+constexpr size_t kOffStatus = 0;          // sticky status word (kvzip_workspace_status)
+constexpr size_t kOffSync = 256;          // barrier count, generation, abort flag
+constexpr size_t kOffH1 = 512;
+constexpr size_t kOffH2 = kOffH1 + kBins1 * 4;
+constexpr size_t kOffH3 = kOffH2 + kBins2 * 4;
+constexpr size_t kOffHeads = kOffH3 + kBins3 * 4;
+
+__host__ __device__ size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+struct Layout {
+  size_t zero_end;    // end of the region zeroed before each launch
+  size_t off_blk;     // blk_cand[kMaxBlocks], blk_tie[kMaxBlocks]
+  size_t off_cand;    // candidate flat indices, one segment per block
+  size_t total;
+};
+
+// Candidate capacity: every block's segment holds its whole range (ranges are
+// multiples of 4 scores), so the buffer never overflows.
+__host__ __device__ Layout layout(int64_t N, int64_t n_heads) {
+  Layout L;
+  L.zero_end = up256(kOffHeads + static_cast<size_t>(n_heads) * 4);
+  L.off_blk = L.zero_end;
+  L.off_cand = L.off_blk + up256(2 * kMaxBlocks * 4);
+  L.total = L.off_cand + up256((static_cast<size_t>(N) + 4 * kMaxBlocks) * 4);
+  return L;
+}
+
+struct Params {
+  const float* s;
+  uint32_t N, n_c, n_heads;
+  uint64_t k;
+  uint8_t* keep;
+  int64_t* offsets;
+  float* threshold;
+  uint8_t* ws;
+  uint32_t* cand;        // base of the candidate buffer
+  uint32_t seg;          // scores per block range (multiple of 4)
+  uint64_t timeout_ns;
+  int vec;               // scores 16-byte aligned: 16-byte loads
+  int vec_keep;          // keep 4-byte aligned: 4-byte mask stores
+};
+
+struct Sync {
+  unsigned int count;
+  unsigned int gen;
+  unsigned int abort;
+};
+
+// Grid barrier with a bounded wait.  Returns false if this block must stop
+// (a wait timed out here or elsewhere).
+__device__ bool grid_barrier(Sync* sy, uint32_t* status, uint64_t timeout_ns) {
+  __shared__ int ok_s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    volatile unsigned int* vgen = &sy->gen;
+    volatile unsigned int* vabort = &sy->abort;
+    const unsigned int g = *vgen;
+    __threadfence();
+    int ok = 1;
+    if (atomicAdd(&sy->count, 1u) == gridDim.x - 1) {
+      atomicExch(&sy->count, 0u);
+      __threadfence();
+      atomicAdd(&sy->gen, 1u);
+    } else {
+      const uint64_t t0 = globaltimer_ns();
+      while (*vgen == g) {
+        if (*vabort) {
+          ok = 0;
+          break;
+        }
+        if (globaltimer_ns() - t0 > timeout_ns) {
+          atomicOr(status, kStatusTimeout);
+          atomicExch(&sy->abort, 1u);
+          ok = 0;
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    __threadfence();
+    ok_s = ok && !*vabort;
+  }
+  __syncthreads();
+  return ok_s != 0;
+}
+
+// Block-wide exclusive scan of one 32-bit value per thread (kThr threads).
+// `tmp` holds kThr/32 words; returns the exclusive prefix and the block total.
+__device__ __forceinline__ uint32_t block_excl(uint32_t v, uint32_t* tmp, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t n = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += n;
+  }
+  if (lane == 31) tmp[warp] = inc;
+  __syncthreads();
+  uint32_t before = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < kThr / 32; ++w) {
+    const uint32_t t = tmp[w];
+    before += (w < warp) ? t : 0u;
+    tot += t;
+  }
+  __syncthreads();
+  *total = tot;
+  return before + inc - v;
+}
+
+// The bin (scanning from the top) that holds the k_rem-th largest element of a
+// histogram with NB bins in global memory; every thread gets the answer.
+template <int NB>
+__device__ void pick_bin(const uint32_t* h, uint64_t k_rem, int* bin_out, uint64_t* above_out) {
+  constexpr int PER = NB / kThr;          // 16, 2 or 1 bins per thread
+  __shared__ unsigned long long wsum[kThr / 32];
+  __shared__ int bin_s;
+  __shared__ unsigned long long above_s;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t c[PER];
+  unsigned long long mine = 0;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {      // thread t owns bins NB-1-PER*t ... descending
+    c[j] = __ldcg(h + (NB - 1 - (PER * threadIdx.x + j)));
+    mine += c[j];
+  }
+  unsigned long long inc = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long n = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += n;
+  }
+  if (lane == 31) wsum[warp] = inc;
+  if (threadIdx.x == 0) bin_s = -1;
+  __syncthreads();
+  unsigned long long base = 0;
+  for (int w = 0; w < warp; ++w) base += wsum[w];
+  const unsigned long long excl = base + inc - mine, incl = base + inc;
+  if (excl < k_rem && k_rem <= incl) {
+    unsigned long long above = excl;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      if (above + c[j] >= k_rem) {
+        bin_s = NB - 1 - (PER * threadIdx.x + j);
+        above_s = above;
+        break;
+      }
+      above += c[j];
+    }
+  }
+  __syncthreads();
+  *bin_out = bin_s;
+  *above_out = above_s;
+  __syncthreads();
+}
+
+// Run-length per-head counting: a thread adds kept scores of head `h` until
+// its flat index crosses into another head, then flushes the count.
+struct HeadCounter {
+  uint32_t h = 0, end = 0, cnt = 0;
+  __device__ __forceinline__ void at(uint32_t f, uint32_t n_c, uint32_t* heads) {
+    if (f >= end) {
+      if (cnt) atomicAdd(heads + h, cnt);
+      cnt = 0;
+      h = f / n_c;
+      end = (h + 1) * n_c;
+    }
+  }
+  __device__ __forceinline__ void flush(uint32_t* heads) {
+    if (cnt) atomicAdd(heads + h, cnt);
+    cnt = 0;
+  }
+};
+
+__global__ void __launch_bounds__(kThr)
+    select_fused_kernel(const Params p) {
+  __shared__ uint32_t h1[kBins1];       // round-1 histogram (32 KB), reused by later rounds
+  __shared__ uint32_t h2[kBins2];
+  __shared__ uint32_t tmp[2 * (kThr / 32)];
+
+  uint32_t* status = reinterpret_cast<uint32_t*>(p.ws + kOffStatus);
+  Sync* sy = reinterpret_cast<Sync*>(p.ws + kOffSync);
+  uint32_t* g1 = reinterpret_cast<uint32_t*>(p.ws + kOffH1);
+  uint32_t* g2 = reinterpret_cast<uint32_t*>(p.ws + kOffH2);
+  uint32_t* g3 = reinterpret_cast<uint32_t*>(p.ws + kOffH3);
+  uint32_t* heads = reinterpret_cast<uint32_t*>(p.ws + kOffHeads);
+  const Layout Lw = layout(p.N, p.n_heads);
+  uint32_t* blk_cand = reinterpret_cast<uint32_t*>(p.ws + Lw.off_blk);
+  uint32_t* blk_tie = blk_cand + kMaxBlocks;
+
+  const uint32_t lo = blockIdx.x * p.seg;
+  const uint32_t hi = min(lo + p.seg, p.N);
+  uint32_t* seg = p.cand + static_cast<size_t>(blockIdx.x) * p.seg;
+  const uint4* s4 = reinterpret_cast<const uint4*>(p.s);
+  const uint32_t* su = reinterpret_cast<const uint32_t*>(p.s);
+  const bool none = p.k == 0;
+
+  // ------------------------------------------------------------ A: round-1 histogram
+  if (!none) {
+    for (int i = threadIdx.x; i < kBins1; i += kThr) h1[i] = 0;
+    __syncthreads();
+    for (uint32_t i0 = lo + 4 * threadIdx.x; i0 < hi; i0 += 2 * kTile) {
+      uint32_t w[8];
+      const uint32_t i1 = i0 + kTile;
+      if (p.vec && i1 + 3 < hi) {
+        const uint4 a = __ldg(s4 + i0 / 4), b = __ldg(s4 + i1 / 4);
+        w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+        w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) atomicAdd(&h1[w[e] >> kShift1], 1u);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const uint32_t f = (e < 4 ? i0 : i1) + (e & 3);
+          if (f < hi) atomicAdd(&h1[__ldg(su + f) >> kShift1], 1u);
+        }
+      }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < kBins1; i += kThr)
+      if (h1[i]) atomicAdd(g1 + i, h1[i]);
+  }
+  if (!grid_barrier(sy, status, p.timeout_ns)) return;
+
+  // ------------------------------------------------------------ B: bin of round 1
+  int b1 = -1;
+  uint64_t k_rem = p.k;
+  if (!none) {
+    uint64_t above;
+    pick_bin<kBins1>(g1, k_rem, &b1, &above);
+    k_rem -= above;
+  }
+
+  // ------------------------------------------------------------ C: mask, candidates, round-2 histogram
+  for (int i = threadIdx.x; i < kBins2; i += kThr) h2[i] = 0;
+  __syncthreads();
+  HeadCounter hc;
+  uint32_t n_cand = 0;   // block-uniform running candidate count
+  const uint32_t ub1 = static_cast<uint32_t>(b1);
+  for (uint32_t i0 = lo + 4 * threadIdx.x, t0 = lo; t0 < hi; i0 += kTile, t0 += kTile) {
+    uint32_t w[4] = {0, 0, 0, 0};
+    const bool full = i0 + 3 < hi;
+    if (p.vec && full) {
+      const uint4 a = __ldcs(s4 + i0 / 4);
+      w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (i0 + e < hi) w[e] = __ldcs(su + i0 + e);
+    }
+    uint32_t km = 0, cm = 0;   // kept / candidate flags, one bit per score
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t d = w[e] >> kShift1;
+      const bool in = i0 + e < hi;
+      km |= static_cast<uint32_t>(in && !none && d > ub1) << e;
+      cm |= static_cast<uint32_t>(in && !none && d == ub1) << e;
+    }
+    // mask bytes: final for every non-candidate, 0 for candidates (set in F)
+    if (p.vec_keep && full) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) word |= ((km >> e) & 1u) << (8 * e);
+      *reinterpret_cast<uint32_t*>(p.keep + i0) = word;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (i0 + e < hi) p.keep[i0 + e] = static_cast<uint8_t>((km >> e) & 1u);
+    }
+    if (km) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if ((km >> e) & 1u) {
+          hc.at(i0 + e, p.n_c, heads);
+          ++hc.cnt;
+        }
+    }
+    // append candidates in flat order
+    uint32_t tot;
+    const uint32_t pos = n_cand + block_excl(__popc(cm), tmp, &tot);
+    if (cm) {
+      uint32_t q = pos;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if ((cm >> e) & 1u) {
+          seg[q++] = i0 + e;
+          atomicAdd(&h2[(w[e] >> kShift2) & (kBins2 - 1)], 1u);
+        }
+    }
+    n_cand += tot;
+  }
+  hc.flush(heads);
+  __syncthreads();
+  for (int i = threadIdx.x; i < kBins2; i += kThr)
+    if (h2[i]) atomicAdd(g2 + i, h2[i]);
+  if (threadIdx.x == 0) blk_cand[blockIdx.x] = n_cand;
+  if (!grid_barrier(sy, status, p.timeout_ns)) return;
+
+  uint32_t tau = 0x7F800000u;
+  uint64_t take_eq = 0;
+  bool rank_ties = false;
+  uint64_t tie_base = 0;
+  if (!none) {
+    // ---------------------------------------------------------- D: round 2, round-3 histogram
+    int b2;
+    uint64_t above;
+    pick_bin<kBins2>(g2, k_rem, &b2, &above);
+    k_rem -= above;
+    const uint32_t pre2 = (ub1 << kShift1) | (static_cast<uint32_t>(b2) << kShift2);
+    uint32_t* h3 = h1;   // reuse
+    for (int i = threadIdx.x; i < kBins3; i += kThr) h3[i] = 0;
+    __syncthreads();
+    for (uint32_t j = threadIdx.x; j < n_cand; j += kThr) {
+      const uint32_t w = __ldg(su + seg[j]);
+      if ((w >> kShift2) == (pre2 >> kShift2)) atomicAdd(&h3[w & (kBins3 - 1)], 1u);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < kBins3; i += kThr)
+      if (h3[i]) atomicAdd(g3 + i, h3[i]);
+    if (!grid_barrier(sy, status, p.timeout_ns)) return;
+
+    // ---------------------------------------------------------- E: threshold, tie ranks
+    int b3;
+    pick_bin<kBins3>(g3, k_rem, &b3, &above);
+    k_rem -= above;
+    tau = pre2 | static_cast<uint32_t>(b3);
+    take_eq = k_rem;                                   // scores equal to tau that are kept
+    const uint64_t n_eq = __ldcg(g3 + b3);
+    rank_ties = take_eq < n_eq;                        // the same decision in every block
+    if (rank_ties) {
+      uint32_t c = 0;
+      for (uint32_t j = threadIdx.x; j < n_cand; j += kThr) c += (__ldg(su + seg[j]) == tau);
+      uint32_t tot;
+      block_excl(c, tmp, &tot);
+      if (threadIdx.x == 0) blk_tie[blockIdx.x] = tot;
+      if (!grid_barrier(sy, status, p.timeout_ns)) return;
+      uint32_t part = 0;
+      for (uint32_t b = threadIdx.x; b < blockIdx.x; b += kThr) part += __ldcg(blk_tie + b);
+      block_excl(part, tmp, &tot);
+      tie_base = tot;
+    }
+
+    // ---------------------------------------------------------- F: kept candidates
+    HeadCounter hf;
+    uint64_t ties_seen = 0;   // block-uniform: ties in earlier candidate tiles of this block
+    for (uint32_t jb = 0; jb < n_cand; jb += kThr) {
+      const uint32_t j = jb + threadIdx.x;
+      const bool in = j < n_cand;
+      const uint32_t f = in ? seg[j] : 0u;
+      const uint32_t w = in ? __ldg(su + f) : 0u;
+      const bool eq = in && w == tau;
+      bool kp = in && (w > tau || (eq && !rank_ties));
+      if (rank_ties) {
+        uint32_t tot;
+        const uint32_t r = block_excl(eq ? 1u : 0u, tmp, &tot);
+        kp = kp || (eq && tie_base + ties_seen + r < take_eq);
+        ties_seen += tot;
+      }
+      if (kp) {
+        p.keep[f] = 1;
+        hf.at(f, p.n_c, heads);
+        ++hf.cnt;
+      }
+    }
+    hf.flush(heads);
+  }
+  if (!grid_barrier(sy, status, p.timeout_ns)) return;
+
+  // ------------------------------------------------------------ G: offsets, threshold
+  if (blockIdx.x != 0) return;
+  unsigned long long carry = 0;
+  for (uint32_t base = 0; base < p.n_heads; base += kThr) {
+    const uint32_t hh = base + threadIdx.x;
+    const uint32_t c = hh < p.n_heads ? __ldcg(heads + hh) : 0u;
+    uint32_t tot;
+    const uint32_t ex = block_excl(c, tmp, &tot);
+    if (hh < p.n_heads) p.offsets[hh] = static_cast<int64_t>(carry + ex);
+    carry += tot;
+  }
+  if (threadIdx.x == 0) {
+    p.offsets[p.n_heads] = static_cast<int64_t>(carry);
+    if (p.threshold) *p.threshold = none ? INFINITY : __uint_as_float(tau);
+  }
+}
+
+std::mutex g_coop_mu;
+int g_coop_blocks[64] = {};   // co-resident blocks per device (0 = not yet queried)
+
+cudaError_t coop_capacity(int* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_coop_mu);
+  if (!g_coop_blocks[dev]) {
+    int sms = 0, per_sm = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_fused_kernel, kThr, 0);
+    if (e != cudaSuccess) return e;
+    g_coop_blocks[dev] = std::max(1, std::min(kMaxBlocks, sms * per_sm));
+  }
+  *out = g_coop_blocks[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+size_t select_fused_ws_bytes(int64_t N, int64_t n_heads) { return layout(N, n_heads).total; }
+
+cudaError_t launch_select_fused(const SelectArgs& a, uint64_t timeout_ns, cudaStream_t s,
+                                int* launches) {
+  int cap = 0;
+  cudaError_t e = coop_capacity(&cap);
+  if (e != cudaSuccess) return e;
+  const int64_t N = a.N;
+  // Blocks: enough to fill the GPU, but no block with less than one tile.
+  const int64_t want = (N + kTile - 1) / kTile;
+  const int P = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(cap, want)));
+  int64_t seg = (N + P - 1) / P;
+  seg = (seg + 3) / 4 * 4;
+  const int P_used = static_cast<int>((N + seg - 1) / seg);
+  const Layout L = layout(N, a.n_heads);
+  uint8_t* ws = static_cast<uint8_t*>(a.ws);
+  e = cudaMemsetAsync(ws + kOffSync, 0, L.zero_end - kOffSync, s);
+  if (e != cudaSuccess) return e;
+  Params p;
+  p.s = a.scores;
+  p.N = static_cast<uint32_t>(N);
+  p.n_c = static_cast<uint32_t>(a.n_c);
+  p.n_heads = static_cast<uint32_t>(a.n_heads);
+  p.k = static_cast<uint64_t>(a.k);
+  p.keep = a.keep;
+  p.offsets = a.offsets;
+  p.threshold = a.threshold;
+  p.ws = ws;
+  p.cand = reinterpret_cast<uint32_t*>(ws + L.off_cand);
+  p.seg = static_cast<uint32_t>(seg);
+  p.timeout_ns = timeout_ns;
+  p.vec = reinterpret_cast<uintptr_t>(a.scores) % 16 == 0 ? 1 : 0;   // ranges start on 4 scores
+  p.vec_keep = reinterpret_cast<uintptr_t>(a.keep) % 4 == 0 ? 1 : 0;
+  void* args[] = {&p};
+  e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(select_fused_kernel),
+                                  dim3(P_used), dim3(kThr), args, 0, s);
+  if (e != cudaSuccess) return e;
+  if (launches) *launches += 1;
+  return cudaSuccess;
+}
+
+}  // namespace kvzip

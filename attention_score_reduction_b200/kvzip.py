@@ -49,6 +49,13 @@ def _load() -> ctypes.CDLL:
         "kvzip_select_workspace_size": (sz, [i64, i64]),
         "kvzip_select": (i32, [vp, i64, i64, i64, vp, vp, vp, vp, sz, vp]),
         "kvzip_select_noalloc": (i32, [vp, i64, i64, i64, vp, vp, vp, vp]),
+        "kvzip_select_shard_bins": (i32, [i32]),
+        "kvzip_select_shard_workspace_size": (sz, [i64, i64]),
+        "kvzip_select_shard_begin": (i32, [i64, vp, sz, vp]),
+        "kvzip_select_shard_hist": (i32, [vp, i64, i32, vp, vp, sz, vp]),
+        "kvzip_select_shard_pick": (i32, [vp, i32, vp, vp, sz, vp]),
+        "kvzip_select_shard_ties": (i32, [vp, i64, vp, vp, sz, vp]),
+        "kvzip_select_shard_mask": (i32, [vp, i64, i64, vp, i32, vp, vp, vp, sz, vp]),
         "kvzip_compact_workspace_size": (sz, [i64, i32]),
         "kvzip_compact": (i32, [vp, vp, vp, vp, i64, i32, i32, vp, vp, vp, vp, sz, vp]),
         "kvzip_head_scores": (i32, [vp, i64, i64, vp, vp]),
@@ -258,12 +265,63 @@ def select(scores: torch.Tensor, k: int, n_heads: int, keep: torch.Tensor | None
     offsets = torch.empty(n_heads + 1, dtype=torch.int64, device=dev) if offsets is None else offsets
     threshold = torch.empty(1, dtype=torch.float32, device=dev) if threshold is None else threshold
     if workspace is None:
-        workspace = torch.empty(max(select_workspace_size(N, n_heads), 256), dtype=torch.uint8,
+        workspace = torch.zeros(max(select_workspace_size(N, n_heads), 256), dtype=torch.uint8,
                                 device=dev)
     s = _lib.kvzip_select(_ptr(scores), N, int(k), int(n_heads), _ptr(keep), _ptr(offsets),
                           _ptr(threshold), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(s, "kvzip_select")
     return keep, offsets, threshold
+
+
+# ---------------------------------------------------------------- sharded selection
+
+def shard_bins(round_: int) -> int:
+    return int(_lib.kvzip_select_shard_bins(int(round_)))
+
+
+def shard_workspace(N_local: int, n_heads_local: int, device=None) -> torch.Tensor:
+    n = int(_lib.kvzip_select_shard_workspace_size(N_local, n_heads_local))
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def shard_begin(k: int, workspace: torch.Tensor, stream=None):
+    _check(_lib.kvzip_select_shard_begin(int(k), _ptr(workspace), workspace.numel(),
+                                         _stream(stream)), "kvzip_select_shard_begin")
+
+
+def shard_hist(scores: torch.Tensor, round_: int, hist: torch.Tensor, workspace: torch.Tensor,
+               stream=None):
+    _dev_contig("scores", scores, torch.float32)
+    _dev_contig("hist", hist, torch.int64)
+    if hist.numel() != shard_bins(round_):
+        raise ValueError("hist must hold kvzip_select_shard_bins(round) counts")
+    _check(_lib.kvzip_select_shard_hist(_ptr(scores), scores.numel(), int(round_), _ptr(hist),
+                                        _ptr(workspace), workspace.numel(), _stream(stream)),
+           "kvzip_select_shard_hist")
+
+
+def shard_pick(hist: torch.Tensor, round_: int, threshold: torch.Tensor | None,
+               workspace: torch.Tensor, stream=None):
+    _dev_contig("hist", hist, torch.int64)
+    _check(_lib.kvzip_select_shard_pick(_ptr(hist), int(round_), _ptr(threshold),
+                                        _ptr(workspace), workspace.numel(), _stream(stream)),
+           "kvzip_select_shard_pick")
+
+
+def shard_ties(scores: torch.Tensor, n_ties: torch.Tensor, workspace: torch.Tensor, stream=None):
+    _dev_contig("n_ties", n_ties, torch.int64)
+    _check(_lib.kvzip_select_shard_ties(_ptr(scores), scores.numel(), _ptr(n_ties),
+                                        _ptr(workspace), workspace.numel(), _stream(stream)),
+           "kvzip_select_shard_ties")
+
+
+def shard_mask(scores: torch.Tensor, n_heads_local: int, tie_counts: torch.Tensor, rank: int,
+               keep: torch.Tensor, offsets: torch.Tensor, workspace: torch.Tensor, stream=None):
+    _dev_contig("tie_counts", tie_counts, torch.int64)
+    _check(_lib.kvzip_select_shard_mask(_ptr(scores), scores.numel(), int(n_heads_local),
+                                        _ptr(tie_counts), int(rank), _ptr(keep), _ptr(offsets),
+                                        _ptr(workspace), workspace.numel(), _stream(stream)),
+           "kvzip_select_shard_mask")
 
 
 # ---------------------------------------------------------------- compaction

@@ -48,7 +48,7 @@ class Compressor:
         N = units * n_c
         self.scores = torch.zeros(units, n_c, dtype=torch.float32, device=self.device)
         self.score_ws = kz.new_context_workspace(units, G, max_n_in, self.device)
-        self.select_ws = torch.empty(max(kz.select_workspace_size(N, units), 256),
+        self.select_ws = torch.zeros(max(kz.select_workspace_size(N, units), 256),
                                      dtype=torch.uint8, device=self.device)
         self.compact_ws = torch.empty(max(kz.compact_workspace_size(units, n_c), 256),
                                       dtype=torch.uint8, device=self.device)
@@ -93,6 +93,9 @@ class Compressor:
         s = kz.workspace_status(self.score_ws, stream)
         if s != kz.OK:
             raise kz.KvzipError(s, "scoring kernels")
+        s = kz.workspace_status(self.select_ws, stream)
+        if s != kz.OK:
+            raise kz.KvzipError(s, "selection kernel")
 
 
 def compress_from_host(comp: Compressor, k_ctx_h, v_h, q_chunks_h, ks_chunks_h, r: float,
@@ -100,14 +103,20 @@ def compress_from_host(comp: Compressor, k_ctx_h, v_h, q_chunks_h, ks_chunks_h, 
     """Upload host inputs, compress, and read the compacted cache back.
 
     k_ctx_h, v_h: pinned host [units][n_c][d]; q_chunks_h / ks_chunks_h: lists of
-    pinned host chunk tensors.  ``dev_bufs`` holds reusable device tensors
-    ("k_ctx", "v", and lists "q", "ks" of per-chunk buffers).  ``host_out``
-    (pinned) receives "k", "v", "pos", "offsets".  Uploads run on a side
-    stream, each chunk's upload recorded by an event the scorer waits on.
+    pinned host chunk tensors (one per chunk, in order).  ``dev_bufs`` holds
+    reusable device tensors: "k_ctx", "v", and lists "q", "ks" of chunk buffers.
+    When the lists are shorter than the chunk list they are used as a ring:
+    chunk c goes into buffer c % len, and its upload waits until the scorer has
+    finished the chunk that last used that buffer.  ``host_out`` (pinned)
+    receives "k", "v", "pos", "offsets".  Uploads run on a side stream, each
+    chunk's upload recorded by an event the scorer waits on.
     Returns (Compressed on the device, host_out, bytes_h2d, bytes_d2h).
     """
     main = torch.cuda.current_stream()
     copy = dev_bufs.setdefault("_copy_stream", torch.cuda.Stream())
+    n_buf = len(dev_bufs["q"])
+    if n_buf == 0 or len(dev_bufs["ks"]) != n_buf or len(q_chunks_h) != len(ks_chunks_h):
+        raise ValueError("need matching lists of chunk inputs and device chunk buffers")
     copy.wait_stream(main)          # device buffers are free once earlier work is done
     h2d = 0
     with torch.cuda.stream(copy):
@@ -116,19 +125,28 @@ def compress_from_host(comp: Compressor, k_ctx_h, v_h, q_chunks_h, ks_chunks_h, 
         h2d += k_ctx_h.numel() * k_ctx_h.element_size() + v_h.numel() * v_h.element_size()
         ev_kv = torch.cuda.Event()
         ev_kv.record(copy)
-        evs = []
-        for qd, ksd, qh, ksh in zip(dev_bufs["q"], dev_bufs["ks"], q_chunks_h, ks_chunks_h):
+    comp.reset()
+    main.wait_event(ev_kv)
+    freed = [None] * n_buf          # event: the scorer is done with this ring slot
+    for c, (qh, ksh) in enumerate(zip(q_chunks_h, ks_chunks_h)):
+        slot = c % n_buf
+        qd, ksd = dev_bufs["q"][slot], dev_bufs["ks"][slot]
+        if qd.shape != qh.shape or ksd.shape != ksh.shape:   # a ragged last chunk
+            qd = qd.view(-1)[:qh.numel()].view(qh.shape)
+            ksd = ksd.view(-1)[:ksh.numel()].view(ksh.shape)
+        with torch.cuda.stream(copy):
+            if freed[slot] is not None:
+                copy.wait_event(freed[slot])
             qd.copy_(qh, non_blocking=True)
             ksd.copy_(ksh, non_blocking=True)
             h2d += qh.numel() * qh.element_size() + ksh.numel() * ksh.element_size()
-            e = torch.cuda.Event()
-            e.record(copy)
-            evs.append(e)
-    comp.reset()
-    main.wait_event(ev_kv)
-    for qd, ksd, e in zip(dev_bufs["q"], dev_bufs["ks"], evs):
-        main.wait_event(e)
+            up = torch.cuda.Event()
+            up.record(copy)
+        main.wait_event(up)
         comp.score_chunk(qd, dev_bufs["k_ctx"], ksd, scale)
+        done = torch.cuda.Event()
+        done.record(main)
+        freed[slot] = done
     kept = comp.select(r)
     k_out, v_out, pos = comp.compact(dev_bufs["k_ctx"], dev_bufs["v"], kept)
     d2h = 0

@@ -73,10 +73,11 @@ def workload(args, rank=0):
     return wl
 
 
-def config_dict(wl, r):
+def config_dict(wl, r, resident=True):
     return {"workload": wl.name, "L": wl.L, "H": wl.H, "G": wl.G, "d": wl.d, "n_c": wl.n_c,
             "chunk": wl.m, "prompt_rows": wl.P, "chunks": wl.n_chunks, "r": r,
             "inputs": "synthetic, seeded; " + _recipe(wl),
+            "chunk_inputs": "resident in HBM" if resident else "drawn on the device per chunk",
             "l2": "inputs larger than L2 (K_ctx alone is %.1f GB per step)"
                   % (wl.units * wl.n_c * wl.d * 2 / 1e9)}
 
@@ -169,6 +170,13 @@ def run_reference(args):
 
 # ----------------------------------------------------------------- our arm
 
+def _resident_bytes(wl):
+    """Device bytes of K_ctx, V and every chunk's Q and K_self."""
+    kv = 2 * wl.units * wl.n_c * wl.d * 2
+    per_in = sum(wl.n_in(c) for c in range(wl.n_chunks))
+    return kv + wl.units * per_in * wl.d * 2 * (wl.G + 1)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -187,9 +195,14 @@ def main():
     wl = workload(args, rank)
     r = args.r if args.r is not None else wl.r[0]
     dev = torch.device("cuda", local)
+    free, total = torch.cuda.mem_get_info(dev)
+    # Chunk inputs stay resident when they fit with room for the outputs;
+    # otherwise each chunk's Q / K_self is drawn on the device just before its
+    # launches, outside the timed events (the 170K Gemma3-12B shape: ~100 GB).
+    resident = _resident_bytes(wl) < 0.7 * total
     k_ctx, v = synth.context_kv(wl, device=dev)
-    chunks = [synth.chunk_qk(wl, c, device=dev) for c in range(wl.n_chunks)]
-    max_n_in = max(q.shape[2] for q, _ in chunks)
+    chunks = [synth.chunk_qk(wl, c, device=dev) for c in range(wl.n_chunks)] if resident else None
+    max_n_in = max(wl.n_in(c) for c in range(wl.n_chunks))
     comp = pipeline.Compressor(wl.units, wl.n_c, wl.d, wl.G, max_n_in, device=dev)
     N = wl.units * wl.n_c
     kept = kz.keep_count(r, N)
@@ -198,6 +211,9 @@ def main():
     pos_out = torch.empty(kept, dtype=torch.int32, device=dev)
     torch.cuda.synchronize()
 
+    def chunk(c):
+        return chunks[c] if resident else synth.chunk_qk(wl, c, device=dev)
+
     stream = torch.cuda.current_stream()
     per_launch = []  # (event before, event after, kernel name, flops) per scorer launch, timed steps
     stage_ev = []
@@ -205,7 +221,8 @@ def main():
     def step(timed: bool):
         comp.reset()
         launches = 0
-        for q, ks in chunks:   # per chunk: pass 1 (row normalisers), then pass 2 (column max)
+        for c in range(wl.n_chunks):   # per chunk: pass 1 (row normalisers), then pass 2 (column max)
+            q, ks = chunk(c)
             f = bu.score_flops(wl.units, wl.G, q.shape[2], wl.n_c, wl.d)
             for which, name in (("lse", "score_pass1_lse"), ("colmax", "score_pass2_colmax")):
                 if timed:
@@ -217,6 +234,7 @@ def main():
                     e1.record(stream)
                     per_launch.append((e0, e1, name,
                                        f["pass1"] if which == "lse" else f["pass2"]))
+            del q, ks
         if timed:
             s0, s1, s2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
             s0.record(stream)
@@ -250,13 +268,24 @@ def main():
     bu.barrier(world)
     comp.check_status()
     clocks = clk.summary()
-    elapsed_ms = bu.max_over_ranks(start.elapsed_time(end), world, dev)
-    ms_per_step = elapsed_ms / args.steps
+    sel = [a.elapsed_time(b) for a, b, _ in stage_ev]
+    cmp = [b.elapsed_time(c) for _, b, c in stage_ev]
+    if resident:
+        step_ms = start.elapsed_time(end) / args.steps
+        timing = "K whole steps between two events on the launching stream"
+    else:
+        step_ms = (sum(a.elapsed_time(b) for a, b, _, _ in per_launch) + sum(sel) + sum(cmp)) / args.steps
+        timing = ("sum of per-launch events (scorer passes, selection, compaction); each chunk's "
+                  "Q / K_self drawn on the device between timed launches")
+    ms_per_step = bu.max_over_ranks(step_ms, world, dev)
     value = world * wl.n_c / (ms_per_step / 1e3)
 
     # per-kernel device times
     peaks = bu.load_peaks(os.path.join(ROOT, "MEASURED_PEAKS.json"))
     peak_tf = peaks["bf16_tflops_sustained"]
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    clock_peak_tf = (bu.clock_peak_tflops(sms, clocks.get("sm_mhz"))
+                     if clocks.get("sm_mhz") else None)
     by_kernel = {}
     for a, b, name, flops in per_launch:
         by_kernel.setdefault(name, []).append((a.elapsed_time(b), flops))
@@ -266,10 +295,10 @@ def main():
         f = sum(fl for _, fl in rows) / len(rows)
         tf = f / (t * 1e-3) / 1e12
         kernels[name] = {"launches_per_step": len(rows) // args.steps, "ms": t,
-                         "tflop_per_launch": f / 1e12, "tflops": tf, "frac_of_peak": tf / peak_tf}
+                         "tflop_per_launch": f / 1e12, "tflops": tf, "frac_of_peak": tf / peak_tf,
+                         "frac_of_burst_peak": tf / peaks["bf16_tflops"],
+                         "frac_of_clock_peak": (tf / clock_peak_tf) if clock_peak_tf else None}
     dominant = max(by_kernel, key=lambda n: sum(ms for ms, _ in by_kernel[n]))
-    sel = [a.elapsed_time(b) for a, b, _ in stage_ev]
-    cmp = [b.elapsed_time(c) for _, b, c in stage_ev]
     # selection / compaction bytes: scores read once + mask written; kept K and V rows
     # read and written once, positions written, mask read once.
     sel_bytes = N * 4 + N
@@ -282,7 +311,11 @@ def main():
                 "unit": "TFLOP/s", "frac": dk["frac_of_peak"],
                 "traffic": NCU_TRAFFIC.get((wl.name, wl.L, dominant)),
                 "peak_source": f"{peaks['source']} bf16 sustained",
-                "flops_per_launch": dk["tflop_per_launch"] * 1e12}
+                "flops_per_launch": dk["tflop_per_launch"] * 1e12,
+                "frac_of_burst_peak": dk["frac_of_burst_peak"],
+                "frac_of_clock_peak": dk["frac_of_clock_peak"],
+                "clock_peak_tflops": clock_peak_tf,
+                "clock_peak_basis": f"{sms} SMs x 8192 dense bf16 flop/clk x median SM clock"}
     kernels.update({
         "select": {"ms": t_sel, "gbs": sel_bytes / (t_sel * 1e-3) / 1e9,
                    "frac_of_hbm": sel_bytes / (t_sel * 1e-3) / 1e9 / peaks["hbm_gbs"]},
@@ -302,18 +335,18 @@ def main():
 
     variants = None
     if not args.no_variants:
-        variants = run_variants(wl, comp, k_ctx, chunks[0], r, dev, peaks)
+        variants = run_variants(wl, comp, k_ctx, chunk(0), r, dev, peaks)
 
     # ------------------------------------------------------------ end to end
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, wl, r, comp, k_ctx, v, chunks, kept, world, dev)
+        e2e = run_e2e(args, wl, r, comp, k_ctx, v, chunk, kept, world, dev, resident)
 
     out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-           "data": "synthetic", "config": config_dict(wl, r), "parallelism":
-           f"{world} independent contexts, one per GPU", "clocks": clocks,
+           "data": "synthetic", "config": config_dict(wl, r, resident), "parallelism":
+           f"{world} independent contexts, one per GPU", "timing": timing, "clocks": clocks,
            "gpu_launches": launches, "roofline": roofline, "kernels": kernels,
            "pct_bf16_tc_peak": kernels["step_pct_bf16_tc_peak"], "e2e": e2e,
            "decode_attention": decode, "variants": variants}
@@ -455,27 +488,41 @@ def _unpin(ts):
         torch.cuda.cudart().cudaHostUnregister(h.data_ptr())
 
 
-def run_e2e(args, wl, r, comp, k_ctx, v, chunks, kept, world, dev):
+def run_e2e(args, wl, r, comp, k_ctx, v, chunk, kept, world, dev, resident):
     """Same step from pinned host memory: uploads, scoring, selection, compaction
     and the read-back of the compacted cache all inside the timed region.
 
     The host holds K_ctx, V and as many distinct chunk inputs as a host-memory
     budget allows (all of them on a single-GPU run with enough RAM); when it
     holds fewer, chunks reuse host buffers cyclically, so every chunk is still
-    uploaded in full each step."""
+    uploaded in full each step.  When the chunk inputs are not resident on the
+    device they stream through a ring of three device buffers."""
     import psutil
     from attention_score_reduction_b200 import pipeline
     steps = args.e2e_steps or max(1, args.steps)
-    per_chunk = sum(t.numel() * t.element_size() for t in chunks[0])
+    q0, ks0 = chunk(0)
+    per_chunk = q0.numel() * q0.element_size() + ks0.numel() * ks0.element_size()
     fixed = 2 * k_ctx.numel() * k_ctx.element_size() + 2 * kept * wl.d * 2
     budget = 0.6 * psutil.virtual_memory().available / world
-    n_host = int(max(1, min(len(chunks), (budget - fixed) // max(per_chunk, 1))))
+    if budget < fixed + per_chunk:
+        return {"skipped": f"host RAM: {fixed / 1e9:.1f} GB of pinned K/V and output needed, "
+                           f"{budget / 1e9:.1f} GB budget"}
+    n_host = int(max(1, min(wl.n_chunks, (budget - fixed) // max(per_chunk, 1))))
     k_h, v_h = _pinned_like(k_ctx), _pinned_like(v)
-    q_h = [_pinned_like(chunks[c][0]) for c in range(n_host)]
-    ks_h = [_pinned_like(chunks[c][1]) for c in range(n_host)]
-    qs = [q_h[c % n_host] for c in range(len(chunks))]
-    kss = [ks_h[c % n_host] for c in range(len(chunks))]
-    bufs = {"k_ctx": k_ctx, "v": v, "q": [q for q, _ in chunks], "ks": [ks for _, ks in chunks]}
+    q_h, ks_h = [], []
+    for c in range(n_host):
+        q, ks = chunk(c)
+        q_h.append(_pinned_like(q))
+        ks_h.append(_pinned_like(ks))
+        del q, ks
+    qs = [q_h[c % n_host] for c in range(wl.n_chunks)]
+    kss = [ks_h[c % n_host] for c in range(wl.n_chunks)]
+    if resident:
+        ring = [chunk(c) for c in range(wl.n_chunks)]
+    else:   # three device slots of the largest chunk's size
+        ring = [(torch.empty_like(q0), torch.empty_like(ks0)) for _ in range(3)]
+    del q0, ks0
+    bufs = {"k_ctx": k_ctx, "v": v, "q": [q for q, _ in ring], "ks": [ks for _, ks in ring]}
     host_out = {"k": torch.empty(kept, wl.d, dtype=torch.bfloat16),
                 "v": torch.empty(kept, wl.d, dtype=torch.bfloat16),
                 "pos": torch.empty(kept, dtype=torch.int32),
@@ -501,7 +548,7 @@ def run_e2e(args, wl, r, comp, k_ctx, v, chunks, kept, world, dev):
     _unpin([k_h, v_h] + q_h + ks_h + list(host_out.values()))
     return {"value": world * wl.n_c / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
             "steps": steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "host_chunk_buffers": n_host}
+            "host_chunk_buffers": n_host, "device_chunk_buffers": len(ring)}
 
 
 if __name__ == "__main__":

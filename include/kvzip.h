@@ -169,7 +169,8 @@ void kvzip_set_test_stall(int on);
  * [0, 1] or N < 0.  r is the KEPT fraction ("30% cache ratio"). */
 int64_t kvzip_keep_count(double r, int64_t N);
 
-/* Bytes of workspace kvzip_select needs. */
+/* Bytes of workspace kvzip_select needs: about 4 * N bytes (a candidate
+ * buffer of flat indices) plus ~40 KB and 4 bytes per head. */
 size_t kvzip_select_workspace_size(int64_t N, int64_t n_heads);
 
 /*
@@ -188,6 +189,14 @@ size_t kvzip_select_workspace_size(int64_t N, int64_t n_heads);
  *             offsets[n_heads] = k.  8-byte aligned.
  *   threshold float out or NULL: the k-th largest score (+inf if k == 0).
  *   N < 2^31.
+ *   workspace >= kvzip_select_workspace_size(N, n_heads) bytes, 256-byte
+ *             aligned.  Its first 4 bytes are a sticky status word, as in the
+ *             scoring workspace: zero it before first use; kvzip_workspace_status
+ *             reads and clears it.
+ *
+ * One kernel launch (cooperative: its blocks wait on one another at bounded
+ * grid barriers; if a wait runs out, the status word records
+ * KVZIP_ERR_TIMEOUT and the mask is incomplete).  The scores are read twice.
  */
 kvzip_status kvzip_select(const float* scores, int64_t N, int64_t k, int64_t n_heads,
                           uint8_t* keep, int64_t* offsets, float* threshold,
@@ -202,10 +211,11 @@ kvzip_status kvzip_select(const float* scores, int64_t N, int64_t k, int64_t n_h
  *
  * Same arguments and results as kvzip_select, but the selection scratch is a
  * library-owned static device array of 1 MiB on every GPU that loads the
- * library (held until the process exits).  It fits problems with
- * kvzip_select_workspace_size(N, n_heads) <= 1 MiB, i.e. roughly
- * n_heads * ceil(n_c / 8192) <= 126000 (all LLaMA3.1-8B / Qwen2.5-14B /
- * Gemma3-12B shapes up to 170K tokens); larger ones return
+ * library (held until the process exits).  It runs the multi-launch radix
+ * selection (eleven small kernels, three when k == 0), whose scratch is
+ * about 40 KB plus 8 bytes per 8192 scores of each head, so it fits problems
+ * with roughly n_heads * ceil(n_c / 8192) <= 126000 (all LLaMA3.1-8B /
+ * Qwen2.5-14B / Gemma3-12B shapes up to 170K tokens); larger ones return
  * KVZIP_ERR_UNSUPPORTED without launching anything.  N must be >= 1.
  *   - The first call on each device looks up the array's device address with
  *     that device current; make that first call before any stream capture.
@@ -217,6 +227,58 @@ kvzip_status kvzip_select(const float* scores, int64_t N, int64_t k, int64_t n_h
 kvzip_status kvzip_select_noalloc(const float* scores, int64_t N, int64_t k, int64_t n_heads,
                                   uint8_t* keep, int64_t* offsets, float* threshold,
                                   void* stream);
+
+/* ------------------------------------------------------- sharded selection */
+
+/*
+ * The same global selection when one context's heads are split across ranks
+ * (one process per GPU, e.g. tensor-parallel serving where every GPU already
+ * holds some KV heads of every layer).  The ranking is global over all L x H x
+ * n_c scores (rebuttal: S has shape L x H x n_c; scime.ai "Measured effects":
+ * non-uniform head budgets need the global ranking), so the ranks exchange
+ * small summaries between the steps below; the caller does the exchange with
+ * its own collectives.  Rank r holds a contiguous run of heads, ranks in
+ * flat-index order (rank 0 the first heads), N_local = n_heads_local * n_c
+ * scores each.  The result equals kvzip_select on the concatenated scores:
+ * each rank gets the keep mask of its own scores and offsets over its own
+ * heads (offsets[n_heads_local] = rows it keeps).
+ *
+ *   ws = this rank's workspace (kvzip_select_shard_workspace_size bytes,
+ *        256-byte aligned); k = the GLOBAL kept count (<= the sum of N_local).
+ *
+ *   kvzip_select_shard_begin(k, ws)
+ *   for round in 0, 1, 2:
+ *     kvzip_select_shard_hist(scores, N_local, round, hist, ws)
+ *         hist: device int64[kvzip_select_shard_bins(round)] out, this rank's
+ *         counts (the call zeroes it first)
+ *     caller: hist <- element-wise SUM of hist over all ranks (all-reduce)
+ *     kvzip_select_shard_pick(hist, round, threshold, ws)
+ *         threshold: device float or NULL, set to the k-th largest score of
+ *         the whole context after round 2
+ *   kvzip_select_shard_ties(scores, N_local, n_ties, ws)
+ *         n_ties: device int64[1] out, this rank's scores equal to the threshold
+ *   caller: tie_counts <- n_ties of every rank, indexed by rank (all-gather)
+ *   kvzip_select_shard_mask(scores, N_local, n_heads_local, tie_counts, rank,
+ *                           keep, offsets, ws)
+ *
+ * Every rank must run every step, in this order, with the same k.  Scores
+ * 16-byte aligned, finite and >= 0; 1 <= N_local < 2^31.  All calls are
+ * asynchronous on `stream`; the caller orders its collectives after them.
+ */
+int kvzip_select_shard_bins(int round);   /* 8192, 1024, 512; 0 for other rounds */
+size_t kvzip_select_shard_workspace_size(int64_t N_local, int64_t n_heads_local);
+kvzip_status kvzip_select_shard_begin(int64_t k, void* workspace, size_t ws_bytes, void* stream);
+kvzip_status kvzip_select_shard_hist(const float* scores, int64_t N_local, int round,
+                                     int64_t* hist, void* workspace, size_t ws_bytes,
+                                     void* stream);
+kvzip_status kvzip_select_shard_pick(const int64_t* hist, int round, float* threshold,
+                                     void* workspace, size_t ws_bytes, void* stream);
+kvzip_status kvzip_select_shard_ties(const float* scores, int64_t N_local, int64_t* n_ties,
+                                     void* workspace, size_t ws_bytes, void* stream);
+kvzip_status kvzip_select_shard_mask(const float* scores, int64_t N_local, int64_t n_heads_local,
+                                     const int64_t* tie_counts, int rank, uint8_t* keep,
+                                     int64_t* offsets, void* workspace, size_t ws_bytes,
+                                     void* stream);
 
 /* --------------------------------------------------------------- compaction */
 

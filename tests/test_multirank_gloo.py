@@ -64,3 +64,57 @@ def test_score_flops_counts_pairs():
     R = 15
     assert f["pass2"] == 2 * 4 * 2 * R * 7
     assert f["pass1"] == 2 * 4 * 2 * (R * 7 + 3 * 5 * 6 // 2)
+
+
+def _shard_worker(rank, world, port, q, heads, n_c, levels, ks):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from attention_score_reduction_b200 import sharded, synth
+        from tests import shard_fake
+        s = synth.random_scores(sum(heads), n_c, seed=7 + levels, levels=levels)
+        h0 = sum(heads[:rank])
+        mine = s[h0:h0 + heads[rank]].contiguous()
+        out = []
+        for k in ks:
+            keep, off, thr = sharded.select_sharded(mine, k, backend=shard_fake)
+            out.append((keep.numpy().copy(), off.numpy().copy(), float(thr.item())))
+        q.put((rank, out))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("heads,n_c,levels", [((3, 5), 300, 0), ((4, 4), 257, 8), ((2, 6), 100, 2),
+                                              ((5, 3), 64, 1)])
+def test_sharded_selection_exchange_matches_global(heads, n_c, levels):
+    """Two gloo ranks, each holding a run of heads (uneven splits), run the
+    sharded selection's exchange (histogram all-reduce per radix round, tie
+    count all-gather); the concatenated masks, the per-rank offsets and the
+    threshold equal the oracle's global selection, including tie-heavy arrays
+    where the ties at the threshold straddle the two ranks."""
+    import numpy as np
+
+    import oracle
+    from attention_score_reduction_b200 import synth
+    N = sum(heads) * n_c
+    ks = [0, 1, oracle.keep_count(0.3, N), oracle.keep_count(0.5, N), N - 1, N]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 30500 + (os.getpid() % 1000) + 7 * levels
+    procs = [ctx.Process(target=_shard_worker, args=(r, 2, port, q, heads, n_c, levels, ks))
+             for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    s = synth.random_scores(sum(heads), n_c, seed=7 + levels, levels=levels).numpy()
+    for i, k in enumerate(ks):
+        keep_ref, off_ref, thr_ref = oracle.select(s.reshape(-1), k, sum(heads))
+        keep = np.concatenate([res[0][i][0], res[1][i][0]])
+        assert np.array_equal(keep, keep_ref), (k, levels)
+        off0, off1 = res[0][i][1], res[1][i][1]
+        assert np.array_equal(off0, off_ref[:heads[0] + 1])
+        assert np.array_equal(off1 + off0[-1], off_ref[heads[0]:])
+        assert res[0][i][2] == res[1][i][2] == thr_ref
