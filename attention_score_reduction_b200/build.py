@@ -17,6 +17,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libkvzip.so")
+LIB_DEBUG = os.path.join(HERE, "libkvzip_debug.so")   # with the device bounds checks
 SOURCES = ["kvzip_api.cu", "score_tc.cu", "score_simt.cu", "select.cu", "select_fused.cu", "compact.cu", "heads.cu", "decode.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -28,19 +29,22 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def _needs_rebuild() -> bool:
-    if not os.path.exists(LIB):
+def _needs_rebuild(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(INCLUDE, "kvzip.h"),
                                                                os.path.abspath(__file__)]
     return any(os.path.getmtime(p) > t for p in deps)
 
 
 def build(force: bool = False, debug: bool = False, verbose: bool = False) -> str:
-    if not force and not debug and not _needs_rebuild():
-        return LIB
-    build_dir = os.path.join(ROOT, "_build")
+    """Compile libkvzip.so (or, with debug=True, libkvzip_debug.so with the
+    device bounds checks) unless it is newer than every source."""
+    lib = LIB_DEBUG if debug else LIB
+    if not force and not _needs_rebuild(lib):
+        return lib
+    build_dir = os.path.join(ROOT, "_build_debug" if debug else "_build")
     os.makedirs(build_dir, exist_ok=True)
     common = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",
                      "-I" + INCLUDE, "-I" + CSRC]
@@ -58,14 +62,14 @@ def build(force: bool = False, debug: bool = False, verbose: bool = False) -> st
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed on {src}")
         objs.append(obj)
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [nvcc()] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs + ["-lrt", "-ldl", "-lpthread"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
         raise RuntimeError("link failed")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
@@ -74,4 +78,4 @@ if __name__ == "__main__":
     ap.add_argument("--verbose", action="store_true", help="print ptxas register/smem usage")
     ap.add_argument("--force", action="store_true")
     a = ap.parse_args()
-    print(build(force=True if (a.force or a.verbose) else False, debug=a.debug, verbose=a.verbose))
+    print(build(force=bool(a.force or a.verbose), debug=a.debug, verbose=a.verbose))

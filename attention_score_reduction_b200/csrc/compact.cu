@@ -114,7 +114,8 @@ __global__ void __launch_bounds__(kCmpThreads)
     const uint32_t rank = before + __popc(m & ((1u << lane) - 1u));
     if (kept) {
       list[rank] = static_cast<int>(j);
-      if (pos_out && out + rank < head_end) pos_out[out + rank] = static_cast<int32_t>(j);
+      if (pos_out && out + rank < head_end && in_bounds(out + rank >= 0))
+        pos_out[out + rank] = static_cast<int32_t>(j);
     }
     __syncthreads();
     // copy the `total` kept rows of this group; ROWS_PER_PASS rows per step
@@ -122,6 +123,8 @@ __global__ void __launch_bounds__(kCmpThreads)
     for (uint32_t r = sub; r < total; r += ROWS_PER_PASS) {
       const int64_t o = out + r;
       if (o >= head_end) break;
+      // destination row inside the packed output, source row inside head h
+      if (!in_bounds(o >= 0 && h < n_heads && list[r] >= j0 && list[r] < j1)) continue;
       const int64_t src = (h * n_c + list[r]) * LPR + col;
       const uint4 kv = ld_stream(k + src);
       const uint4 vv = ld_stream(v + src);
@@ -134,6 +137,8 @@ __global__ void __launch_bounds__(kCmpThreads)
 }
 
 }  // namespace
+
+cudaError_t bounds_flag_compact(unsigned int* out) { return take_bounds_flag(out); }
 
 size_t compact_ws_bytes(int64_t n_heads, int n_c) {
   const int64_t nblk = n_heads * cmp_segs(n_c);

@@ -99,7 +99,9 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS)
   const int h = blockIdx.y, s = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t base = offsets[h];
-  const int64_t len = offsets[h + 1] - base;
+  int64_t len = offsets[h + 1] - base;
+  // the head's kept rows must lie inside the packed cache; otherwise read none
+  if (!in_bounds(base >= 0 && len >= 0 && base + len <= offsets[gridDim.y])) len = 0;
   const int64_t r0 = base + len * s / S, r1 = base + len * (s + 1) / S;
   uint8_t* ks = dsm + warp * 2 * Cfg::BATCH_BYTES;
   uint8_t* vs = ks + Cfg::BATCH_BYTES;
@@ -329,6 +331,8 @@ cudaError_t launch_decode_d(const DecodeArgs& a, cudaStream_t st, int* launches)
 }
 
 }  // namespace
+
+cudaError_t bounds_flag_decode(unsigned int* out) { return take_bounds_flag(out); }
 
 int decode_splits(int64_t n_heads) {
   // about two CTAs (one per SM at a time) per SM of a 148-SM B200 in total,

@@ -36,6 +36,7 @@ const char* kvzip_status_string(kvzip_status s) {
     case KVZIP_ERR_UNSUPPORTED: return "unsupported shape or dtype";
     case KVZIP_ERR_CUDA: return "CUDA error";
     case KVZIP_ERR_TIMEOUT: return "kernel pipeline wait timed out";
+    case KVZIP_ERR_BOUNDS: return "debug bounds check failed";
   }
   return "unknown status";
 }
@@ -45,6 +46,28 @@ void kvzip_set_wait_timeout_ns(uint64_t ns) {
 }
 
 void kvzip_set_test_stall(int on) { g_test_stall.store(on ? 1 : 0); }
+
+int kvzip_debug_checks(void) {
+#ifdef KVZIP_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+kvzip_status kvzip_debug_bounds_status(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return KVZIP_ERR_CUDA;
+  unsigned int any = 0;
+  cudaError_t (*const files[])(unsigned int*) = {
+      kvzip::bounds_flag_score, kvzip::bounds_flag_select, kvzip::bounds_flag_select_fused,
+      kvzip::bounds_flag_compact, kvzip::bounds_flag_decode};
+  for (auto take : files) {
+    unsigned int f = 0;
+    if (take(&f) != cudaSuccess) return KVZIP_ERR_CUDA;
+    any |= f;
+  }
+  return any ? KVZIP_ERR_BOUNDS : KVZIP_OK;
+}
 
 /* Number of kernel launches the most recent successful call enqueued (testing aid). */
 int kvzip_last_launch_count(void) { return g_last_launches.load(); }

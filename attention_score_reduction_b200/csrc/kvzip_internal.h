@@ -123,4 +123,38 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, int* launches);
 // Records the launch count of an accepted call (read by kvzip_last_launch_count).
 void note_launches(int launches);
 
+// Debug bounds checks.  Built with -DKVZIP_DEBUG, the kernels that read or
+// write through computed indices test each index against the extent of its
+// buffer first; a failed test sets this file's flag word and the access is
+// skipped (no trap, no fault), so that kvzip_debug_bounds_status can report it
+// after the call.  In normal builds in_bounds() is always true and the tests
+// compile away.  Every kernel file includes this header and so has its own
+// flag word; bounds_flag_*() read and clear them (host, synchronous).
+#ifdef KVZIP_DEBUG
+static __device__ unsigned int g_bounds_flag;
+__device__ __forceinline__ bool in_bounds(bool ok) {
+  if (!ok) atomicOr(&g_bounds_flag, 1u);
+  return ok;
+}
+static inline cudaError_t take_bounds_flag(unsigned int* out) {
+  unsigned int v = 0;
+  const unsigned int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_bounds_flag, sizeof(v));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_bounds_flag, &zero, sizeof(zero));
+  *out = v;
+  return e;
+}
+#else
+__device__ __forceinline__ bool in_bounds(bool) { return true; }
+static inline cudaError_t take_bounds_flag(unsigned int* out) {
+  *out = 0;
+  return cudaSuccess;
+}
+#endif
+cudaError_t bounds_flag_score(unsigned int* out);
+cudaError_t bounds_flag_select(unsigned int* out);
+cudaError_t bounds_flag_select_fused(unsigned int* out);
+cudaError_t bounds_flag_compact(unsigned int* out);
+cudaError_t bounds_flag_decode(unsigned int* out);
+
 }  // namespace kvzip

@@ -235,19 +235,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = (it / STAGES) & 1;
         if (!wait_one(&b_empty[s], ph ^ 1, ctl)) break;
         if (PASS2 && !wait_one(&l_empty[s], ph ^ 1, ctl)) break;
-        mbar_arrive_expect_tx(&b_full[s], Lay::B_BYTES + (PASS2 ? Lay::L_BYTES : 0));
         const void* map = &bmap0;
         int row = it * BN;
         if (!PASS2 && it >= n_kt_ctx) {
           map = &bmap1;
           row = (it - n_kt_ctx) * BN;
         }
+        // pass 2: the tile's BN normalisers must lie inside the unit's padded rows
+        const uint32_t l_bytes = (PASS2 && in_bounds(row + BN <= p.R_pad)) ? Lay::L_BYTES : 0u;
+        mbar_arrive_expect_tx(&b_full[s], Lay::B_BYTES + l_bytes);
         uint8_t* dst = smem + Lay::OFF_B + s * Lay::B_BYTES;
         for (int kb = 0; kb < KB; ++kb)
           tma_load_3d(dst + kb * Lay::B_KB_BYTES, map, &b_full[s], kb * 64, row, b);
-        if (PASS2)  // the row normalisers of this query tile ride on the same barrier
+        if (l_bytes)  // the row normalisers of this query tile ride on the same barrier
           bulk_load(smem + Lay::OFF_L + s * Lay::L_BYTES,
-                    p.lse2 + static_cast<size_t>(b) * p.R_pad + row, Lay::L_BYTES, &b_full[s]);
+                    p.lse2 + static_cast<size_t>(b) * p.R_pad + row, l_bytes, &b_full[s]);
         issued = it + 1;
       }
       // Drain: every copy this CTA started must land before shared memory is released.
@@ -513,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (par == 1) xchg->x = best;
         named_barrier_sync(1 + t, 2 * kBM);
-        if (par == 0 && !*abort_flag && arow < p.n_c) {
+        if (par == 0 && !*abort_flag && arow < p.n_c && in_bounds(b < static_cast<int>(gridDim.y))) {
           float* dst = p.scores + static_cast<size_t>(b) * p.n_c + arow;
           if (SUM)
             *dst += best + xchg->x;
@@ -544,6 +546,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------ host side
+
+cudaError_t bounds_flag_score(unsigned int* out) { return take_bounds_flag(out); }
 
 template <int D>
 static cudaError_t launch_tc(const ScoreArgs& a, cudaStream_t s, int* launches) {

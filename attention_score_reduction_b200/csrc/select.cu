@@ -305,6 +305,8 @@ __global__ void __launch_bounds__(kSelThreads)
   __shared__ uint32_t red[kSelThreads / 32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint32_t kept = 0;
+  // mask words of this block stay inside head h's n_c bytes
+  if (!in_bounds(j0 + 4 * n4 <= n_c)) return;
   if (none) {
     for (int64_t i = threadIdx.x; i < n4; i += kSelThreads) k4[i] = 0u;
   } else if (!rank_ties) {   // every score >= tau is kept
@@ -430,7 +432,7 @@ __global__ void __launch_bounds__(kSelThreads)
       tie_before += total;
       __syncthreads();
     }
-    if (in) kb[j] = k ? 1 : 0;
+    if (in && in_bounds(j < n_c)) kb[j] = k ? 1 : 0;
     kept += k;
   }
   kept = __reduce_add_sync(0xffffffffu, kept);
@@ -680,6 +682,8 @@ int hist_grid(int64_t N) {
 }
 
 }  // namespace
+
+cudaError_t bounds_flag_select(unsigned int* out) { return take_bounds_flag(out); }
 
 int shard_bins(int round) { return (round >= 0 && round <= 2) ? hist_bins(round) : 0; }
 

@@ -215,16 +215,16 @@ __device__ void pick_bin(const uint32_t* h, uint64_t k_rem, int* bin_out, uint64
 // its flat index crosses into another head, then flushes the count.
 struct HeadCounter {
   uint32_t h = 0, end = 0, cnt = 0;
-  __device__ __forceinline__ void at(uint32_t f, uint32_t n_c, uint32_t* heads) {
+  __device__ __forceinline__ void at(uint32_t f, uint32_t n_c, uint32_t n_heads,
+                                     uint32_t* heads) {
     if (f >= end) {
-      if (cnt) atomicAdd(heads + h, cnt);
-      cnt = 0;
+      flush(n_heads, heads);
       h = f / n_c;
       end = (h + 1) * n_c;
     }
   }
-  __device__ __forceinline__ void flush(uint32_t* heads) {
-    if (cnt) atomicAdd(heads + h, cnt);
+  __device__ __forceinline__ void flush(uint32_t n_heads, uint32_t* heads) {
+    if (cnt && in_bounds(h < n_heads)) atomicAdd(heads + h, cnt);
     cnt = 0;
   }
 };
@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(kThr)
       cm |= static_cast<uint32_t>(in && !none && d == ub1) << e;
     }
     // mask bytes: final for every non-candidate, 0 for candidates (set in F)
-    if (p.vec_keep && full) {
+    if (p.vec_keep && full && in_bounds(i0 + 3 < p.N)) {
       uint32_t word = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) word |= ((km >> e) & 1u) << (8 * e);
@@ -328,7 +328,7 @@ __global__ void __launch_bounds__(kThr)
 #pragma unroll
       for (int e = 0; e < 4; ++e)
         if ((km >> e) & 1u) {
-          hc.at(i0 + e, p.n_c, heads);
+          hc.at(i0 + e, p.n_c, p.n_heads, heads);
           ++hc.cnt;
         }
     }
@@ -340,13 +340,15 @@ __global__ void __launch_bounds__(kThr)
 #pragma unroll
       for (int e = 0; e < 4; ++e)
         if ((cm >> e) & 1u) {
-          seg[q++] = i0 + e;
+          // inside this block's segment (its range length) of the candidate buffer
+          if (in_bounds(q < hi - lo)) seg[q] = i0 + e;
+          ++q;
           atomicAdd(&h2[(w[e] >> kShift2) & (kBins2 - 1)], 1u);
         }
     }
     n_cand += tot;
   }
-  hc.flush(heads);
+  hc.flush(p.n_heads, heads);
   __syncthreads();
   for (int i = threadIdx.x; i < kBins2; i += kThr)
     if (h2[i]) atomicAdd(g2 + i, h2[i]);
@@ -413,13 +415,13 @@ __global__ void __launch_bounds__(kThr)
         kp = kp || (eq && tie_base + ties_seen + r < take_eq);
         ties_seen += tot;
       }
-      if (kp) {
+      if (kp && in_bounds(f >= lo && f < hi)) {
         p.keep[f] = 1;
-        hf.at(f, p.n_c, heads);
+        hf.at(f, p.n_c, p.n_heads, heads);
         ++hf.cnt;
       }
     }
-    hf.flush(heads);
+    hf.flush(p.n_heads, heads);
   }
   if (!grid_barrier(sy, status, p.timeout_ns)) return;
 
@@ -464,6 +466,8 @@ cudaError_t coop_capacity(int* out) {
 }  // namespace
 
 size_t select_fused_ws_bytes(int64_t N, int64_t n_heads) { return layout(N, n_heads).total; }
+
+cudaError_t bounds_flag_select_fused(unsigned int* out) { return take_bounds_flag(out); }
 
 cudaError_t launch_select_fused(const SelectArgs& a, uint64_t timeout_ns, cudaStream_t s,
                                 int* launches) {

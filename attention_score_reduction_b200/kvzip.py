@@ -12,9 +12,11 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libkvzip.so")
+# KVZIP_LIBRARY selects another build of the same ABI (e.g. libkvzip_debug.so,
+# the build with device bounds checks); by default the in-tree libkvzip.so.
+LIB_PATH = os.environ.get("KVZIP_LIBRARY") or os.path.join(_HERE, "libkvzip.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = 0, 1, 2, 3, 4, 5
 BF16, F32 = 0, 1
 
 
@@ -67,6 +69,8 @@ def _load() -> ctypes.CDLL:
         "kvzip_decode_workspace_size": (sz, [i64, i32, i32]),
         "kvzip_decode_attention": (i32, [vp, vp, vp, vp, i64, i32, i32, f32, vp, vp, sz, vp]),
         "kvzip_last_launch_count": (i32, []),
+        "kvzip_debug_checks": (i32, []),
+        "kvzip_debug_bounds_status": (i32, []),
         "kvzip_status_string": (ctypes.c_char_p, [i32]),
     }
     for name, (res, args) in sig.items():

@@ -46,7 +46,8 @@ typedef enum {
   KVZIP_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, short workspace */
   KVZIP_ERR_UNSUPPORTED = 2,   /* well-formed but not implemented (e.g. head dim 64) */
   KVZIP_ERR_CUDA = 3,          /* a CUDA runtime/driver call or launch failed */
-  KVZIP_ERR_TIMEOUT = 4        /* a kernel gave up waiting on its own pipeline */
+  KVZIP_ERR_TIMEOUT = 4,       /* a kernel gave up waiting on its own pipeline */
+  KVZIP_ERR_BOUNDS = 5         /* debug builds: an index failed its bounds check */
 } kvzip_status;
 
 typedef enum {
@@ -387,6 +388,22 @@ kvzip_status kvzip_head_scores(const float* scores, int64_t n_heads, int64_t n_c
 /* Number of kernel launches the most recent accepted call enqueued
  * (process-wide; for tests and launch accounting). */
 int kvzip_last_launch_count(void);
+
+/* ------------------------------------------------------------ debug build */
+
+/* 1 if this library was built with the debug bounds checks (libkvzip_debug.so,
+ * `python -m attention_score_reduction_b200.build --debug`), else 0.  In that
+ * build the kernels that read or write through computed indices (compaction,
+ * both selection paths, the scorer's normaliser tiles and score updates, the
+ * decode row ranges) test every such index against its buffer first; a failed
+ * test skips the access and sets a flag (no trap, no fault).  Normal builds
+ * carry no checks. */
+int kvzip_debug_checks(void);
+
+/* Synchronise the current device, then report whether any bounds check failed
+ * since the previous call (KVZIP_ERR_BOUNDS) or not (KVZIP_OK), and clear the
+ * flags.  Always KVZIP_OK in normal builds. */
+kvzip_status kvzip_debug_bounds_status(void);
 
 /* Static, human-readable name of a status code. */
 const char* kvzip_status_string(kvzip_status s);

@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(kz):
 
 
 def test_status_strings(kz):
-    for s in range(5):
+    for s in range(6):
         assert kz.status_string(s)
     assert kz.status_string(99) == "unknown status"
 
