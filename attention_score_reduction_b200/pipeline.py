@@ -40,16 +40,27 @@ class Compressor:
 
     units = L * H (layer-major), n_c context keys per unit, head dim d, G
     query heads per KV head, max_n_in = largest chunk (prompt + context rows).
+
+    With a process group (``group``), this rank holds ``units`` of the
+    context's ``units_global`` units, ranks in flat-index order; scoring and
+    compaction stay local and the selection ranks all units_global * n_c scores
+    together through ``sharded.select_sharded``.
     """
 
-    def __init__(self, units: int, n_c: int, d: int, G: int, max_n_in: int, device="cuda"):
+    def __init__(self, units: int, n_c: int, d: int, G: int, max_n_in: int, device="cuda",
+                 group=None, units_global: int | None = None):
         self.units, self.n_c, self.d, self.G, self.max_n_in = units, n_c, d, G, max_n_in
         self.device = torch.device(device)
+        self.group = group
+        self.units_global = units_global or units
         N = units * n_c
         self.scores = torch.zeros(units, n_c, dtype=torch.float32, device=self.device)
         self.score_ws = kz.new_context_workspace(units, G, max_n_in, self.device)
-        self.select_ws = torch.zeros(max(kz.select_workspace_size(N, units), 256),
-                                     dtype=torch.uint8, device=self.device)
+        if group is None:
+            self.select_ws = torch.zeros(max(kz.select_workspace_size(N, units), 256),
+                                         dtype=torch.uint8, device=self.device)
+        else:
+            self.select_ws = kz.shard_workspace(N, units, self.device)
         self.compact_ws = torch.empty(max(kz.compact_workspace_size(units, n_c), 256),
                                       dtype=torch.uint8, device=self.device)
         self.keep = torch.empty(N, dtype=torch.uint8, device=self.device)
@@ -64,12 +75,28 @@ class Compressor:
         kz.score_chunk(q, k_ctx, k_self, self.scores, self.score_ws, scale, stream)
         self.launches += kz.last_launch_count()
 
+    def keep_capacity(self, r: float) -> int:
+        """Rows this rank's compacted cache can need: the kept count itself on
+        one GPU; with shards, at most the global count and at most its scores."""
+        k = kz.keep_count(r, self.units_global * self.n_c)
+        return k if self.group is None else min(k, self.scores.numel())
+
     def select(self, r: float, stream=None) -> int:
-        kept = kz.keep_count(r, self.scores.numel())
-        kz.select(self.scores.view(-1), kept, self.units, self.keep, self.offsets, self.threshold,
-                  self.select_ws, stream)
-        self.launches += kz.last_launch_count()
-        return kept
+        """Global top-r selection; returns the kept count (global on one GPU,
+        this rank's capacity bound with shards: offsets[-1] holds its count)."""
+        if self.group is None:
+            kept = kz.keep_count(r, self.scores.numel())
+            kz.select(self.scores.view(-1), kept, self.units, self.keep, self.offsets,
+                      self.threshold, self.select_ws, stream)
+            self.launches += kz.last_launch_count()
+            return kept
+        from . import sharded
+        k = kz.keep_count(r, self.units_global * self.n_c)
+        sharded.select_sharded(self.scores, k, self.group, workspace=self.select_ws,
+                               keep=self.keep, offsets=self.offsets, threshold=self.threshold,
+                               stream=stream)
+        self.launches += 13   # begin, 3 x (histogram, pick), tie count, five-kernel mask
+        return self.keep_capacity(r)
 
     def compact(self, k_ctx, v, kept: int, k_out=None, v_out=None, pos_out=None, stream=None):
         out = kz.compact(k_ctx, v, self.keep, self.offsets, kept, k_out, v_out, pos_out,
@@ -93,9 +120,10 @@ class Compressor:
         s = kz.workspace_status(self.score_ws, stream)
         if s != kz.OK:
             raise kz.KvzipError(s, "scoring kernels")
-        s = kz.workspace_status(self.select_ws, stream)
-        if s != kz.OK:
-            raise kz.KvzipError(s, "selection kernel")
+        if self.group is None:
+            s = kz.workspace_status(self.select_ws, stream)
+            if s != kz.OK:
+                raise kz.KvzipError(s, "selection kernel")
 
 
 def compress_from_host(comp: Compressor, k_ctx_h, v_h, q_chunks_h, ks_chunks_h, r: float,
@@ -148,6 +176,8 @@ def compress_from_host(comp: Compressor, k_ctx_h, v_h, q_chunks_h, ks_chunks_h, 
         done.record(main)
         freed[slot] = done
     kept = comp.select(r)
+    if comp.group is not None:    # this rank's share of the global count (one small read)
+        kept = int(comp.offsets[-1])
     k_out, v_out, pos = comp.compact(dev_bufs["k_ctx"], dev_bufs["v"], kept)
     d2h = 0
     if host_out is not None:
