@@ -482,14 +482,6 @@ SelWs carve(void* ws, int64_t nblk) {
 
 }  // namespace
 
-// Per-head (uniform budget) workspace: one state and one set of histograms per head.
-size_t per_head_ws_bytes(int64_t n_heads, int64_t n_c) {
-  const int64_t nblk = n_heads * segs_per_head(n_c);
-  return align_up(static_cast<size_t>(n_heads) * sizeof(SelState), 256) +
-         align_up(static_cast<size_t>(n_heads) * kHistTotal * 4, 256) +
-         2 * align_up(static_cast<size_t>(nblk) * 4, 256);
-}
-
 size_t select_multipass_ws_bytes(int64_t N, int64_t n_heads) {
   const int64_t n_c = n_heads > 0 ? N / n_heads : 0;
   const int64_t nblk = n_heads * segs_per_head(n_c);
@@ -554,62 +546,6 @@ cudaError_t launch_select_empty(int64_t* offsets, int64_t n_heads, float* thresh
                                 cudaStream_t s, int* launches) {
   sel_empty<<<1, 256, 0, s>>>(offsets, n_heads, threshold);
   if (launches) *launches += 1;
-  return cudaGetLastError();
-}
-
-size_t select_per_head_ws_bytes(int64_t n_heads, int64_t n_c) {
-  return per_head_ws_bytes(n_heads, n_c);
-}
-
-// Uniform head budgets: the same radix selection run for every head at once
-// (grid dimension = head), k_per_head pairs kept in each.
-cudaError_t launch_select_per_head(const SelectArgs& a, cudaStream_t s, int* launches) {
-  const bool vec = use_vec(a);
-  const int64_t segs = segs_per_head(a.n_c);
-  const int64_t nblk = a.n_heads * segs;
-  uint8_t* p = static_cast<uint8_t*>(a.ws);
-  SelState* st = reinterpret_cast<SelState*>(p);
-  p += align_up(static_cast<size_t>(a.n_heads) * sizeof(SelState), 256);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(p);
-  p += align_up(static_cast<size_t>(a.n_heads) * kHistTotal * 4, 256);
-  uint32_t* blk_cnt = reinterpret_cast<uint32_t*>(p);
-  p += align_up(static_cast<size_t>(nblk) * 4, 256);
-  uint32_t* blk_eq = reinterpret_cast<uint32_t*>(p);
-  const unsigned H = static_cast<unsigned>(a.n_heads);
-  int n = 0;
-  sel_init<<<H, 1024, 0, s>>>(st, hist, static_cast<unsigned long long>(a.k), nullptr);
-  ++n;
-  if (a.k > 0) {
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t want = (a.n_c / 4 + kHistThreads - 1) / kHistThreads;
-    const int64_t cap = std::max<int64_t>(1, 4LL * sms / a.n_heads);
-    const dim3 grid(static_cast<unsigned>(std::max<int64_t>(1, std::min(want, cap))), H);
-    sel_hist<0><<<grid, kHistThreads, 0, s>>>(a.scores, a.n_c, st, hist);
-    sel_pick<0><<<H, kPickThreads, 0, s>>>(st, hist, nullptr);
-    sel_hist<1><<<grid, kHistThreads, 0, s>>>(a.scores, a.n_c, st, hist);
-    sel_pick<1><<<H, kPickThreads, 0, s>>>(st, hist, nullptr);
-    sel_hist<2><<<grid, kHistThreads, 0, s>>>(a.scores, a.n_c, st, hist);
-    sel_pick<2><<<H, kPickThreads, 0, s>>>(st, hist, nullptr);
-    if (vec)
-      sel_eqcount_v<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs,
-                                                                       st, blk_eq, 1);
-    else
-      sel_eqcount<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs,
-                                                                     st, blk_eq, 1);
-    sel_scan_blocks<<<H, kPickThreads, 0, s>>>(blk_eq, segs, st, 1);
-    n += 8;
-  }
-  if (vec)
-    sel_mask_v<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs, st,
-                                                                  blk_eq, a.keep, blk_cnt, 1);
-  else
-    sel_mask<<<static_cast<unsigned>(nblk), kSelThreads, 0, s>>>(a.scores, a.n_c, segs, st,
-                                                                blk_eq, a.keep, blk_cnt, 1);
-  sel_offsets<<<1, kPickThreads, 0, s>>>(blk_cnt, a.n_heads, segs, a.offsets);
-  n += 2;
-  if (launches) *launches += n;
   return cudaGetLastError();
 }
 

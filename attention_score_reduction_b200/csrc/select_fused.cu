@@ -166,8 +166,9 @@ __device__ __forceinline__ uint32_t block_excl(uint32_t v, uint32_t* tmp, uint32
 }
 
 // The bin (scanning from the top) that holds the k_rem-th largest element of a
-// histogram with NB bins in global memory; every thread gets the answer.
-template <int NB>
+// histogram with NB bins (in global memory, merged by other blocks, or in this
+// block's shared memory); every thread gets the answer.
+template <int NB, bool SHARED = false>
 __device__ void pick_bin(const uint32_t* h, uint64_t k_rem, int* bin_out, uint64_t* above_out) {
   constexpr int PER = NB / kThr;          // 16, 2 or 1 bins per thread
   __shared__ unsigned long long wsum[kThr / 32];
@@ -178,7 +179,8 @@ __device__ void pick_bin(const uint32_t* h, uint64_t k_rem, int* bin_out, uint64
   unsigned long long mine = 0;
 #pragma unroll
   for (int j = 0; j < PER; ++j) {      // thread t owns bins NB-1-PER*t ... descending
-    c[j] = __ldcg(h + (NB - 1 - (PER * threadIdx.x + j)));
+    const int bin = NB - 1 - (PER * threadIdx.x + j);
+    c[j] = SHARED ? h[bin] : __ldcg(h + bin);
     mine += c[j];
   }
   unsigned long long inc = mine;
@@ -442,6 +444,140 @@ __global__ void __launch_bounds__(kThr)
   }
 }
 
+// Uniform head budgets (scime.ai summary, "Measured effects": the weaker
+// alternative to the global ranking): keep the k largest scores inside every
+// head, lowest position first among equal scores.  One block per head runs the
+// same phases as select_fused_kernel on its own n_c scores with block-level
+// synchronisation only: histogram (read 1), bin of round 1, final mask bytes
+// and candidates in position order (read 2), rounds 2 and 3 and the tie ranks
+// on the candidates, then the kept candidates.  offsets[h] = h * k.
+__global__ void __launch_bounds__(kThr)
+    select_per_head_kernel(const float* __restrict__ s, uint32_t n_c, uint32_t n_heads,
+                           uint32_t k, uint8_t* keep, int64_t* offsets, uint32_t* cand,
+                           int vec, int vec_keep) {
+  __shared__ uint32_t h1[kBins1];
+  __shared__ uint32_t h2[kBins2];
+  __shared__ uint32_t tmp[2 * (kThr / 32)];
+  const uint32_t head = blockIdx.x;
+  const size_t lo = static_cast<size_t>(head) * n_c;
+  const float* sh = s + lo;
+  uint8_t* kh = keep + lo;
+  uint32_t* seg = cand + lo;
+  const uint4* s4 = reinterpret_cast<const uint4*>(sh);
+  const uint32_t* su = reinterpret_cast<const uint32_t*>(sh);
+  const bool none = k == 0;
+  // rows of this head start on 16 bytes only when n_c is a multiple of 4
+  const bool v4 = vec && (n_c % 4 == 0);
+  const bool k4 = vec_keep && (n_c % 4 == 0);
+  if (threadIdx.x == 0) {
+    offsets[head] = static_cast<int64_t>(head) * k;
+    if (head == n_heads - 1) offsets[n_heads] = static_cast<int64_t>(n_heads) * k;
+  }
+
+  int b1 = -1;
+  uint64_t k_rem = k;
+  if (!none) {
+    for (int i = threadIdx.x; i < kBins1; i += kThr) h1[i] = 0;
+    __syncthreads();
+    for (uint32_t i0 = 4 * threadIdx.x; i0 < n_c; i0 += kTile) {
+      if (v4 && i0 + 3 < n_c) {
+        const uint4 a = __ldg(s4 + i0 / 4);
+        atomicAdd(&h1[a.x >> kShift1], 1u);
+        atomicAdd(&h1[a.y >> kShift1], 1u);
+        atomicAdd(&h1[a.z >> kShift1], 1u);
+        atomicAdd(&h1[a.w >> kShift1], 1u);
+      } else {
+        for (uint32_t f = i0; f < i0 + 4 && f < n_c; ++f) atomicAdd(&h1[__ldg(su + f) >> kShift1], 1u);
+      }
+    }
+    __syncthreads();
+    uint64_t above;
+    pick_bin<kBins1, true>(h1, k_rem, &b1, &above);
+    k_rem -= above;
+  }
+  const uint32_t ub1 = static_cast<uint32_t>(b1);
+  for (int i = threadIdx.x; i < kBins2; i += kThr) h2[i] = 0;
+  __syncthreads();
+  uint32_t n_cand = 0;
+  for (uint32_t i0 = 4 * threadIdx.x, t0 = 0; t0 < n_c; i0 += kTile, t0 += kTile) {
+    uint32_t w[4] = {0, 0, 0, 0};
+    const bool full = i0 + 3 < n_c;
+    if (v4 && full) {
+      const uint4 a = __ldcs(s4 + i0 / 4);
+      w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (i0 + e < n_c) w[e] = __ldcs(su + i0 + e);
+    }
+    uint32_t km = 0, cm = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t d = w[e] >> kShift1;
+      const bool in = i0 + e < n_c;
+      km |= static_cast<uint32_t>(in && !none && d > ub1) << e;
+      cm |= static_cast<uint32_t>(in && !none && d == ub1) << e;
+    }
+    if (k4 && full) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) word |= ((km >> e) & 1u) << (8 * e);
+      *reinterpret_cast<uint32_t*>(kh + i0) = word;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (i0 + e < n_c) kh[i0 + e] = static_cast<uint8_t>((km >> e) & 1u);
+    }
+    uint32_t tot;
+    uint32_t q = n_cand + block_excl(__popc(cm), tmp, &tot);
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if ((cm >> e) & 1u) {
+        if (in_bounds(q < n_c)) seg[q] = i0 + e;
+        ++q;
+        atomicAdd(&h2[(w[e] >> kShift2) & (kBins2 - 1)], 1u);
+      }
+    n_cand += tot;
+  }
+  __syncthreads();
+  if (none) return;
+  int b2;
+  uint64_t above;
+  pick_bin<kBins2, true>(h2, k_rem, &b2, &above);
+  k_rem -= above;
+  const uint32_t pre2 = (ub1 << kShift1) | (static_cast<uint32_t>(b2) << kShift2);
+  uint32_t* h3 = h1;
+  for (int i = threadIdx.x; i < kBins3; i += kThr) h3[i] = 0;
+  __syncthreads();
+  for (uint32_t j = threadIdx.x; j < n_cand; j += kThr) {
+    const uint32_t w = __ldg(su + seg[j]);
+    if ((w >> kShift2) == (pre2 >> kShift2)) atomicAdd(&h3[w & (kBins3 - 1)], 1u);
+  }
+  __syncthreads();
+  int b3;
+  pick_bin<kBins3, true>(h3, k_rem, &b3, &above);
+  k_rem -= above;
+  const uint32_t tau = pre2 | static_cast<uint32_t>(b3);
+  const uint64_t take_eq = k_rem;
+  const bool rank_ties = take_eq < h3[b3];
+  uint64_t ties_seen = 0;
+  for (uint32_t jb = 0; jb < n_cand; jb += kThr) {
+    const uint32_t j = jb + threadIdx.x;
+    const bool in = j < n_cand;
+    const uint32_t f = in ? seg[j] : 0u;
+    const uint32_t w = in ? __ldg(su + f) : 0u;
+    const bool eq = in && w == tau;
+    bool kp = in && (w > tau || (eq && !rank_ties));
+    if (rank_ties) {
+      uint32_t tot;
+      const uint32_t r = block_excl(eq ? 1u : 0u, tmp, &tot);
+      kp = kp || (eq && ties_seen + r < take_eq);
+      ties_seen += tot;
+    }
+    if (kp && in_bounds(f < n_c)) kh[f] = 1;
+  }
+}
+
 std::mutex g_coop_mu;
 int g_coop_blocks[64] = {};   // co-resident blocks per device (0 = not yet queried)
 
@@ -466,6 +602,20 @@ cudaError_t coop_capacity(int* out) {
 }  // namespace
 
 size_t select_fused_ws_bytes(int64_t N, int64_t n_heads) { return layout(N, n_heads).total; }
+
+size_t select_per_head_ws_bytes(int64_t n_heads, int64_t n_c) {
+  return up256(static_cast<size_t>(n_heads) * static_cast<size_t>(n_c) * 4);
+}
+
+cudaError_t launch_select_per_head(const SelectArgs& a, cudaStream_t s, int* launches) {
+  select_per_head_kernel<<<static_cast<unsigned>(a.n_heads), kThr, 0, s>>>(
+      a.scores, static_cast<uint32_t>(a.n_c), static_cast<uint32_t>(a.n_heads),
+      static_cast<uint32_t>(a.k), a.keep, a.offsets, static_cast<uint32_t*>(a.ws),
+      reinterpret_cast<uintptr_t>(a.scores) % 16 == 0 ? 1 : 0,
+      reinterpret_cast<uintptr_t>(a.keep) % 4 == 0 ? 1 : 0);
+  if (launches) *launches += 1;
+  return cudaGetLastError();
+}
 
 cudaError_t bounds_flag_select_fused(unsigned int* out) { return take_bounds_flag(out); }
 
