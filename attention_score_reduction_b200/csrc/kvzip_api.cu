@@ -242,7 +242,8 @@ kvzip_status kvzip_select(const float* scores, int64_t N, int64_t k, int64_t n_h
   a.ws = workspace;
   a.ws_bytes = ws_bytes;
   int launches = 0;
-  cudaError_t e = kvzip::launch_select_fused(a, g_timeout_ns.load(), s, &launches);
+  cudaError_t e =
+      kvzip::launch_select_fused(a, g_timeout_ns.load(), g_test_stall.load(), s, &launches);
   if (e == cudaSuccess) g_last_launches.store(launches);
   return from_cuda(e);
 }

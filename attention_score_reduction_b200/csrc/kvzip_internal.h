@@ -51,8 +51,8 @@ struct SelectArgs {
 };
 // One cooperative launch, two reads of the scores (kvzip_select).
 size_t select_fused_ws_bytes(int64_t N, int64_t n_heads);
-cudaError_t launch_select_fused(const SelectArgs& a, uint64_t timeout_ns, cudaStream_t s,
-                                int* launches);
+cudaError_t launch_select_fused(const SelectArgs& a, uint64_t timeout_ns, int test_stall,
+                                cudaStream_t s, int* launches);
 // Multi-launch radix select with a small workspace (kvzip_select_noalloc and the
 // sharded selection).
 size_t select_multipass_ws_bytes(int64_t N, int64_t n_heads);

@@ -95,6 +95,7 @@ struct Params {
   uint64_t timeout_ns;
   int vec;               // scores 16-byte aligned: 16-byte loads
   int vec_keep;          // keep 4-byte aligned: 4-byte mask stores
+  int test_stall;        // test hook: block 0 never reaches a barrier, so the others time out
 };
 
 struct Sync {
@@ -253,6 +254,7 @@ __global__ void __launch_bounds__(kThr)
   const uint4* s4 = reinterpret_cast<const uint4*>(p.s);
   const uint32_t* su = reinterpret_cast<const uint32_t*>(p.s);
   const bool none = p.k == 0;
+  if (p.test_stall && blockIdx.x == 0) return;
 
   // ------------------------------------------------------------ A: round-1 histogram
   if (!none) {
@@ -619,8 +621,8 @@ cudaError_t launch_select_per_head(const SelectArgs& a, cudaStream_t s, int* lau
 
 cudaError_t bounds_flag_select_fused(unsigned int* out) { return take_bounds_flag(out); }
 
-cudaError_t launch_select_fused(const SelectArgs& a, uint64_t timeout_ns, cudaStream_t s,
-                                int* launches) {
+cudaError_t launch_select_fused(const SelectArgs& a, uint64_t timeout_ns, int test_stall,
+                                cudaStream_t s, int* launches) {
   int cap = 0;
   cudaError_t e = coop_capacity(&cap);
   if (e != cudaSuccess) return e;
@@ -650,6 +652,7 @@ cudaError_t launch_select_fused(const SelectArgs& a, uint64_t timeout_ns, cudaSt
   p.timeout_ns = timeout_ns;
   p.vec = reinterpret_cast<uintptr_t>(a.scores) % 16 == 0 ? 1 : 0;   // ranges start on 4 scores
   p.vec_keep = reinterpret_cast<uintptr_t>(a.keep) % 4 == 0 ? 1 : 0;
+  p.test_stall = test_stall;
   void* args[] = {&p};
   e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(select_fused_kernel),
                                   dim3(P_used), dim3(kThr), args, 0, s);

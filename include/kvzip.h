@@ -158,10 +158,12 @@ kvzip_status kvzip_workspace_status(void* workspace, void* stream);
 void kvzip_set_wait_timeout_ns(uint64_t ns);
 
 /* Test hook for the timeout path: while on (nonzero), the bf16 scoring
- * kernels' loader warp issues no copies, so every pipeline wait in them runs
- * out after the wait timeout and the call reports KVZIP_ERR_TIMEOUT through
- * kvzip_workspace_status.  Nothing faults or hangs.  Process-wide; applies to
- * launches enqueued after the call.  Leave off in normal use. */
+ * kernels' loader warp issues no copies, and the first block of kvzip_select's
+ * kernel returns before its first grid barrier, so the waits in them run out
+ * after the wait timeout and the call reports KVZIP_ERR_TIMEOUT through
+ * kvzip_workspace_status (on the scoring or selection workspace).  Nothing
+ * faults or hangs.  Process-wide; applies to launches enqueued after the call.
+ * Leave off in normal use. */
 void kvzip_set_test_stall(int on);
 
 /* ---------------------------------------------------------------- selection */

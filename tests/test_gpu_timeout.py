@@ -52,3 +52,33 @@ def test_timeout_reported_and_context_survives(kz):
     oracle.score_chunk(q.double().numpy(), k.double().numpy(), ks.double().numpy(), want)
     got = S.cpu().double().numpy()
     assert float(np.max(np.abs(got - want) / want)) <= 2e-3
+
+
+def test_selection_grid_barrier_timeout_reported_and_next_call_exact(kz):
+    """The selection kernel's blocks meet at grid barriers whose waits are
+    bounded.  With the test hook on, its first block returns before the first
+    barrier, so every other block's wait runs out (10 ms here): the status word
+    of the selection workspace reports KVZIP_ERR_TIMEOUT and the kernel ends.
+    With the hook off the same call on the same workspace is bit-exact."""
+    from attention_score_reduction_b200 import synth
+    n_heads, n_c = 64, 8192                      # 524288 scores: well over one block
+    s = synth.random_scores(n_heads, n_c, seed=3).reshape(-1).cuda()
+    k = kz.keep_count(0.3, s.numel())
+    ws = torch.zeros(kz.select_workspace_size(s.numel(), n_heads), dtype=torch.uint8,
+                     device="cuda")
+    kz.set_wait_timeout_ns(10_000_000)
+    kz.set_test_stall(True)
+    try:
+        kz.select(s, k, n_heads, workspace=ws)
+        status = kz.workspace_status(ws)
+    finally:
+        kz.set_test_stall(False)
+        kz.set_wait_timeout_ns(0)
+    assert status == kz.ERR_TIMEOUT
+    assert kz.workspace_status(ws) == kz.OK      # reading clears the status
+    keep, off, thr = kz.select(s, k, n_heads, workspace=ws)
+    assert kz.workspace_status(ws) == kz.OK
+    keep_ref, off_ref, thr_ref = oracle.select(s.cpu().numpy(), k, n_heads)
+    assert np.array_equal(keep.cpu().numpy(), keep_ref)
+    assert np.array_equal(off.cpu().numpy(), off_ref)
+    assert float(thr.item()) == thr_ref
