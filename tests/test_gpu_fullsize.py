@@ -92,3 +92,29 @@ def test_fullsize_select_and_compact(kz, full):
             assert torch.equal(ko[a:b], k_ctx[h].index_select(0, idx))
             assert torch.equal(vo[a:b], v[h].index_select(0, idx))
         assert ko.shape[0] == k
+
+
+def test_fullsize_row_normalisers_every_row_tile(kz, full):
+    """Pass 1 at full size, every one of the 8256 query rows of sampled units:
+    the row normalisers (log-sum-exp over 131072 context keys and the row's
+    causal self keys) against the oracle's, for units in the middle of the
+    launch grid.  This covers every 256-row CTA tile of the unit, including the
+    ones in the middle of the row grid and the ragged last tile (rows 8192 to
+    8255).  A normaliser error of e shifts every probability of its row by a
+    factor exp(e), so the bound is the score tolerance itself."""
+    from attention_score_reduction_b200 import synth
+    wl, k_ctx, _ = full
+    q, ks = synth.chunk_qk(wl, 31, device=k_ctx.device)
+    S = torch.zeros(wl.units, wl.n_c, device=k_ctx.device)
+    ws = kz.new_score_workspace(wl.units, wl.G, q.shape[2])
+    kz.score_chunk(q, k_ctx, ks, S, ws, which="lse")
+    assert kz.workspace_status(ws) == kz.OK
+    lse = kz.read_lse(ws, wl.units, wl.G, q.shape[2]).cpu().double().numpy()
+    f = lambda t: t.double().numpy()  # noqa: E731
+    for b in (37, 200):
+        k64, ks64 = f(k_ctx[b].cpu()), f(ks[b].cpu())
+        want = np.concatenate([oracle.unit_chunk_scores(f(q[b, g:g + 1].cpu()), k64, ks64)[1]
+                               for g in range(wl.G)])
+        assert want.shape == (8256,)
+        err = np.abs(lse[b] - want)
+        assert float(err.max()) <= RTOL, (b, float(err.max()), int(err.argmax()))
