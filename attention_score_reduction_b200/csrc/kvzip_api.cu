@@ -256,7 +256,7 @@ size_t kvzip_select_shard_workspace_size(int64_t N_local, int64_t n_heads_local)
 }
 
 static bool shard_args_ok(const float* scores, int64_t N_local, const void* ws, size_t ws_bytes) {
-  return N_local > 0 && N_local < (int64_t{1} << 31) && scores && aligned(scores, 16) && ws &&
+  return N_local > 0 && N_local < (int64_t{1} << 31) && scores && aligned(scores, 4) && ws &&
          aligned(ws, 256) && ws_bytes >= kvzip::select_multipass_ws_bytes(1, 1);
 }
 

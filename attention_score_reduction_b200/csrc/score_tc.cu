@@ -340,14 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t acc_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                 Lay::ACC0 + (t * 2 + par) * BN;
       if (!PASS2) {
-        // ---------------- pass 1: log-sum-exp over the row (this parity's tiles)
-        // l = sum over the tiles seen so far of 2^(c*s - m).  The reference m is
-        // set exactly from the row's first non-empty chunk and then only moves
-        // in whole steps of 64 when l grows past 2^64, so no chunk needs its own
-        // maximum.  A chunk whose sum reaches 2^100 (a logit far above m; also
-        // inf or NaN) is redone exactly: new maximum, rescaled l.  Since m is
-        // always at or below an element already summed, l >= 1 and terms that
-        // flush to zero below 2^-126 are negligible.
+        // ---------------- pass 1: online log-sum-exp over the row (this parity's tiles)
         const int i_row = arow % p.n_in;
         float m = -INFINITY, l = 0.f;
 #pragma unroll 1
@@ -376,78 +369,43 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int j = 0; j < CH; ++j)
                 if (j > lim) v[j] = -INFINITY;
             }
-            bool exact = (m == -INFINITY);
-            if (!exact) {
-              // x = c*s - m in packed pairs; of every 8 pairs, kPolyPairs take 2^x
-              // on the FMA pipe (x clamped to [-125, 126] by a saturating FMA) and
-              // the rest on the MUFU unit (inf above 128, 0 below -126).
-              const float2 c2 = make_float2(c, c);
-              const float2 nm2 = make_float2(-m, -m);
-              const float cs = c * (1.f / kSatSpan), bs = (125.f - m) * (1.f / kSatSpan);
-              float2 acc[4];
+            // chunk maximum, 8 independent chains
+            float mx[8];
 #pragma unroll
-              for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
+            for (int k = 0; k < 8; ++k) mx[k] = fmaxf(v[2 * k], v[2 * k + 1]);
 #pragma unroll
-              for (int j = 0; j < CH; j += 16) {
+            for (int j = 16; j < CH; j += 16) {
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                  float2 e;
-                  if (q < kPolyPairs) {
-                    e = exp2_poly_sat2(make_float2(fma_sat(v[j + 2 * q], cs, bs),
-                                                   fma_sat(v[j + 2 * q + 1], cs, bs)));
-                  } else {
-                    const float2 x = ffma2(make_float2(v[j + 2 * q], v[j + 2 * q + 1]), c2, nm2);
-                    e.x = ex2_approx(x.x);
-                    e.y = ex2_approx(x.y);
-                  }
-                  acc[q & 3] = fadd2(acc[q & 3], e);
-                }
-              }
-              const float2 s4 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
-              const float sum = s4.x + s4.y;
-              if (sum < 0x1p100f) {
-                l += sum;
-                if (l > 0x1p64f) {
-                  m += 64.f;
-                  l *= 0x1p-64f;
-                }
-              } else {
-                exact = true;
-              }
+              for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], v[j + 2 * k], v[j + 2 * k + 1]);
             }
-            if (exact) {
-              // chunk maximum, 8 independent chains
-              float mx[8];
+            const float mxa = fmax3(mx[0], mx[1], mx[2]), mxb = fmax3(mx[3], mx[4], mx[5]);
+            const float m_new = fmaxf(m, fmax3(mxa, mxb, fmaxf(mx[6], mx[7])) * c);
+            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+            // x = c*s - m in packed pairs; of every 8 pairs, kPolyPairs take 2^x on
+            // the FMA pipe and the rest on the MUFU unit.
+            const float2 c2 = make_float2(c, c);
+            const float2 nm2 = make_float2(-m_use, -m_use);
+            float2 acc[4];
 #pragma unroll
-              for (int k = 0; k < 8; ++k) mx[k] = fmaxf(v[2 * k], v[2 * k + 1]);
+            for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
 #pragma unroll
-              for (int j = 16; j < CH; j += 16) {
+            for (int j = 0; j < CH; j += 16) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], v[j + 2 * k], v[j + 2 * k + 1]);
-              }
-              const float mxa = fmax3(mx[0], mx[1], mx[2]), mxb = fmax3(mx[3], mx[4], mx[5]);
-              const float m_new = fmaxf(m, fmax3(mxa, mxb, fmaxf(mx[6], mx[7])) * c);
-              const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-              const float2 c2 = make_float2(c, c);
-              const float2 nm2 = make_float2(-m_use, -m_use);
-              float2 acc[4];
-#pragma unroll
-              for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
-#pragma unroll
-              for (int j = 0; j < CH; j += 16) {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                  const float2 x = ffma2(make_float2(v[j + 2 * q], v[j + 2 * q + 1]), c2, nm2);
-                  float2 e;
+              for (int q = 0; q < 8; ++q) {
+                const float2 x = ffma2(make_float2(v[j + 2 * q], v[j + 2 * q + 1]), c2, nm2);
+                float2 e;
+                if (q < kPolyPairs) {
+                  e = exp2_poly2(x);
+                } else {
                   e.x = ex2_approx(x.x);
                   e.y = ex2_approx(x.y);
-                  acc[q & 3] = fadd2(acc[q & 3], e);
                 }
+                acc[q & 3] = fadd2(acc[q & 3], e);
               }
-              const float2 s4 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
-              l = fmaf(l, ex2_approx(m - m_use), s4.x + s4.y);
-              m = m_new;
             }
+            const float2 s4 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+            l = fmaf(l, ex2_approx(m - m_use), s4.x + s4.y);
+            m = m_new;
           }
         }
         // merge the two parities' (m, l) of this row; parity 0 writes lse2

@@ -571,7 +571,8 @@ __global__ void __launch_bounds__(kHistThreads)
   __shared__ uint32_t h[NB];
   for (int i = threadIdx.x; i < NB; i += blockDim.x) h[i] = 0;
   __syncthreads();
-  if (!st->keep_none) hist_count<PASS>(s, N, st->prefix, true, h);
+  const bool vec = reinterpret_cast<uintptr_t>(s) % 16 == 0;   // 16-byte loads when aligned
+  if (!st->keep_none) hist_count<PASS>(s, N, st->prefix, vec, h);
   __syncthreads();
   for (int i = threadIdx.x; i < NB; i += blockDim.x)
     if (h[i]) atomicAdd(out + i, static_cast<unsigned long long>(h[i]));

@@ -166,6 +166,161 @@ __device__ __forceinline__ uint32_t block_excl(uint32_t v, uint32_t* tmp, uint32
   return before + inc - v;
 }
 
+// The same for two words per thread in one pass (one pair of barriers).
+__device__ __forceinline__ void block_excl2(uint32_t v0, uint32_t v1, uint32_t* tmp,
+                                            uint32_t* ex0, uint32_t* ex1, uint32_t* tot0,
+                                            uint32_t* tot1) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t a = v0, b = v1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t na = __shfl_up_sync(0xffffffffu, a, o);
+    const uint32_t nb = __shfl_up_sync(0xffffffffu, b, o);
+    if (lane >= o) {
+      a += na;
+      b += nb;
+    }
+  }
+  if (lane == 31) {
+    tmp[warp] = a;
+    tmp[kThr / 32 + warp] = b;
+  }
+  __syncthreads();
+  uint32_t ba = 0, bb = 0, ta = 0, tb = 0;
+#pragma unroll
+  for (int w = 0; w < kThr / 32; ++w) {
+    const uint32_t xa = tmp[w], xb = tmp[kThr / 32 + w];
+    ba += (w < warp) ? xa : 0u;
+    bb += (w < warp) ? xb : 0u;
+    ta += xa;
+    tb += xb;
+  }
+  __syncthreads();
+  *ex0 = ba + a - v0;
+  *ex1 = bb + b - v1;
+  *tot0 = ta;
+  *tot1 = tb;
+}
+
+// Round-1 histogram of the top 13 bits of the scores [lo, hi) of s (indices
+// relative to s) into shared memory: four 16-byte loads in flight per thread.
+__device__ __forceinline__ void hist_top(const float* __restrict__ s, uint32_t lo, uint32_t hi,
+                                         bool vec, uint32_t* h1) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(s);
+  const uint32_t* su = reinterpret_cast<const uint32_t*>(s);
+  for (uint32_t g0 = lo; g0 < hi; g0 += 4 * kTile) {
+    const uint32_t i0 = g0 + 4 * threadIdx.x;
+    if (vec && i0 + 3 * kTile + 3 < hi) {
+      uint4 a[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) a[q] = __ldg(s4 + (i0 + q * kTile) / 4);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        atomicAdd(&h1[a[q].x >> kShift1], 1u);
+        atomicAdd(&h1[a[q].y >> kShift1], 1u);
+        atomicAdd(&h1[a[q].z >> kShift1], 1u);
+        atomicAdd(&h1[a[q].w >> kShift1], 1u);
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t f = i0 + q * kTile + e;
+          if (f < hi) atomicAdd(&h1[__ldg(su + f) >> kShift1], 1u);
+        }
+    }
+  }
+}
+
+// Second pass over the scores [lo, hi) of s, four tiles of kTile per step
+// (four 16-byte loads in flight per thread): the final mask byte of every
+// score outside bin b1 (kept iff its bin is above b1; 0 for candidates, set
+// later), the candidates' indices appended to seg in index order (positions
+// from one block scan of packed per-tile counts), their round-2 digits
+// histogrammed into h2, and on_kept(f) for every kept score (in increasing f
+// per thread).  Indices are relative to s; returns the block's candidate count.
+template <class OnKept>
+__device__ uint32_t mask_pass(const float* __restrict__ s, uint32_t lo, uint32_t hi, uint32_t b1,
+                              bool none, bool vec, bool vec_keep, uint8_t* keep, uint32_t* seg,
+                              uint32_t seg_cap, uint32_t* h2, uint32_t* tmp, OnKept on_kept) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(s);
+  const uint32_t* su = reinterpret_cast<const uint32_t*>(s);
+  uint32_t n_cand = 0;   // block-uniform
+  for (uint32_t g0 = lo; g0 < hi; g0 += 4 * kTile) {
+    uint32_t w[4][4];
+    uint32_t i0[4];
+    bool full[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      i0[q] = g0 + q * kTile + 4 * threadIdx.x;
+      full[q] = i0[q] + 3 < hi;
+      if (vec && full[q]) {
+        const uint4 a = __ldcs(s4 + i0[q] / 4);
+        w[q][0] = a.x;
+        w[q][1] = a.y;
+        w[q][2] = a.z;
+        w[q][3] = a.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) w[q][e] = (i0[q] + e < hi) ? __ldcs(su + i0[q] + e) : 0u;
+      }
+    }
+    uint32_t km[4], cm[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      km[q] = cm[q] = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t d = w[q][e] >> kShift1;
+        const bool in = i0[q] + e < hi && !none;
+        km[q] |= static_cast<uint32_t>(in && d > b1) << e;
+        cm[q] |= static_cast<uint32_t>(in && d == b1) << e;
+      }
+      if (vec_keep && full[q]) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) word |= ((km[q] >> e) & 1u) << (8 * e);
+        *reinterpret_cast<uint32_t*>(keep + i0[q]) = word;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (i0[q] + e < hi) keep[i0[q] + e] = static_cast<uint8_t>((km[q] >> e) & 1u);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if ((km[q] >> e) & 1u) on_kept(i0[q] + e);
+    }
+    // candidate positions: counts of tiles 0/1 and 2/3 packed in 16-bit halves
+    // (a tile has at most kTile = 2048 candidates, so the halves never carry)
+    uint32_t ex01, ex23, t01, t23;
+    block_excl2(__popc(cm[0]) | (__popc(cm[1]) << 16), __popc(cm[2]) | (__popc(cm[3]) << 16),
+                tmp, &ex01, &ex23, &t01, &t23);
+    uint32_t base[4], pos[4];
+    base[0] = n_cand;
+    base[1] = base[0] + (t01 & 0xFFFFu);
+    base[2] = base[1] + (t01 >> 16);
+    base[3] = base[2] + (t23 & 0xFFFFu);
+    pos[0] = base[0] + (ex01 & 0xFFFFu);
+    pos[1] = base[1] + (ex01 >> 16);
+    pos[2] = base[2] + (ex23 & 0xFFFFu);
+    pos[3] = base[3] + (ex23 >> 16);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t x = pos[q];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if ((cm[q] >> e) & 1u) {
+          if (in_bounds(x < seg_cap)) seg[x] = i0[q] + e;
+          ++x;
+          atomicAdd(&h2[(w[q][e] >> kShift2) & (kBins2 - 1)], 1u);
+        }
+    }
+    n_cand = base[3] + (t23 >> 16);
+  }
+  return n_cand;
+}
+
 // The bin (scanning from the top) that holds the k_rem-th largest element of a
 // histogram with NB bins (in global memory, merged by other blocks, or in this
 // block's shared memory); every thread gets the answer.
@@ -214,29 +369,46 @@ __device__ void pick_bin(const uint32_t* h, uint64_t k_rem, int* bin_out, uint64
   __syncthreads();
 }
 
-// Run-length per-head counting: a thread adds kept scores of head `h` until
-// its flat index crosses into another head, then flushes the count.
+// Per-head kept counts.  A thread visits its kept scores in increasing flat
+// order, so it adds up a run for one head and only flushes when its index
+// crosses into another head.  Flushes go to a shared-memory window of
+// kHeadWin heads starting at the block's first head (a block's range covers
+// a few heads unless heads are very short), and the block adds the window to
+// the global counts once at the end; heads past the window go to global
+// memory directly.
+constexpr int kHeadWin = 64;
 struct HeadCounter {
   uint32_t h = 0, end = 0, cnt = 0;
-  __device__ __forceinline__ void at(uint32_t f, uint32_t n_c, uint32_t n_heads,
-                                     uint32_t* heads) {
+  uint32_t h_lo, n_c, n_heads;
+  uint32_t* win;      // shared [kHeadWin]
+  uint32_t* heads;    // global [n_heads]
+  __device__ HeadCounter(uint32_t h_lo_, uint32_t n_c_, uint32_t n_heads_, uint32_t* win_,
+                         uint32_t* heads_)
+      : h_lo(h_lo_), n_c(n_c_), n_heads(n_heads_), win(win_), heads(heads_) {}
+  __device__ __forceinline__ void add(uint32_t f) {
     if (f >= end) {
-      flush(n_heads, heads);
+      flush();
       h = f / n_c;
       end = (h + 1) * n_c;
     }
+    ++cnt;
   }
-  __device__ __forceinline__ void flush(uint32_t n_heads, uint32_t* heads) {
-    if (cnt && in_bounds(h < n_heads)) atomicAdd(heads + h, cnt);
+  __device__ __forceinline__ void flush() {
+    if (!cnt) return;
+    if (h - h_lo < static_cast<uint32_t>(kHeadWin))
+      atomicAdd(win + (h - h_lo), cnt);
+    else if (in_bounds(h < n_heads))
+      atomicAdd(heads + h, cnt);
     cnt = 0;
   }
 };
 
-__global__ void __launch_bounds__(kThr)
+__global__ void __launch_bounds__(kThr, 2)
     select_fused_kernel(const Params p) {
   __shared__ uint32_t h1[kBins1];       // round-1 histogram (32 KB), reused by later rounds
   __shared__ uint32_t h2[kBins2];
   __shared__ uint32_t tmp[2 * (kThr / 32)];
+  __shared__ uint32_t win[kHeadWin];
 
   uint32_t* status = reinterpret_cast<uint32_t*>(p.ws + kOffStatus);
   Sync* sy = reinterpret_cast<Sync*>(p.ws + kOffSync);
@@ -251,32 +423,16 @@ __global__ void __launch_bounds__(kThr)
   const uint32_t lo = blockIdx.x * p.seg;
   const uint32_t hi = min(lo + p.seg, p.N);
   uint32_t* seg = p.cand + static_cast<size_t>(blockIdx.x) * p.seg;
-  const uint4* s4 = reinterpret_cast<const uint4*>(p.s);
   const uint32_t* su = reinterpret_cast<const uint32_t*>(p.s);
   const bool none = p.k == 0;
   if (p.test_stall && blockIdx.x == 0) return;
+  for (int i = threadIdx.x; i < kHeadWin; i += kThr) win[i] = 0;
 
   // ------------------------------------------------------------ A: round-1 histogram
   if (!none) {
     for (int i = threadIdx.x; i < kBins1; i += kThr) h1[i] = 0;
     __syncthreads();
-    for (uint32_t i0 = lo + 4 * threadIdx.x; i0 < hi; i0 += 2 * kTile) {
-      uint32_t w[8];
-      const uint32_t i1 = i0 + kTile;
-      if (p.vec && i1 + 3 < hi) {
-        const uint4 a = __ldg(s4 + i0 / 4), b = __ldg(s4 + i1 / 4);
-        w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-        w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) atomicAdd(&h1[w[e] >> kShift1], 1u);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const uint32_t f = (e < 4 ? i0 : i1) + (e & 3);
-          if (f < hi) atomicAdd(&h1[__ldg(su + f) >> kShift1], 1u);
-        }
-      }
-    }
+    hist_top(p.s, lo, hi, p.vec != 0, h1);
     __syncthreads();
     for (int i = threadIdx.x; i < kBins1; i += kThr)
       if (h1[i]) atomicAdd(g1 + i, h1[i]);
@@ -295,64 +451,12 @@ __global__ void __launch_bounds__(kThr)
   // ------------------------------------------------------------ C: mask, candidates, round-2 histogram
   for (int i = threadIdx.x; i < kBins2; i += kThr) h2[i] = 0;
   __syncthreads();
-  HeadCounter hc;
-  uint32_t n_cand = 0;   // block-uniform running candidate count
   const uint32_t ub1 = static_cast<uint32_t>(b1);
-  for (uint32_t i0 = lo + 4 * threadIdx.x, t0 = lo; t0 < hi; i0 += kTile, t0 += kTile) {
-    uint32_t w[4] = {0, 0, 0, 0};
-    const bool full = i0 + 3 < hi;
-    if (p.vec && full) {
-      const uint4 a = __ldcs(s4 + i0 / 4);
-      w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-    } else {
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (i0 + e < hi) w[e] = __ldcs(su + i0 + e);
-    }
-    uint32_t km = 0, cm = 0;   // kept / candidate flags, one bit per score
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint32_t d = w[e] >> kShift1;
-      const bool in = i0 + e < hi;
-      km |= static_cast<uint32_t>(in && !none && d > ub1) << e;
-      cm |= static_cast<uint32_t>(in && !none && d == ub1) << e;
-    }
-    // mask bytes: final for every non-candidate, 0 for candidates (set in F)
-    if (p.vec_keep && full && in_bounds(i0 + 3 < p.N)) {
-      uint32_t word = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) word |= ((km >> e) & 1u) << (8 * e);
-      *reinterpret_cast<uint32_t*>(p.keep + i0) = word;
-    } else {
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (i0 + e < hi) p.keep[i0 + e] = static_cast<uint8_t>((km >> e) & 1u);
-    }
-    if (km) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if ((km >> e) & 1u) {
-          hc.at(i0 + e, p.n_c, p.n_heads, heads);
-          ++hc.cnt;
-        }
-    }
-    // append candidates in flat order
-    uint32_t tot;
-    const uint32_t pos = n_cand + block_excl(__popc(cm), tmp, &tot);
-    if (cm) {
-      uint32_t q = pos;
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if ((cm >> e) & 1u) {
-          // inside this block's segment (its range length) of the candidate buffer
-          if (in_bounds(q < hi - lo)) seg[q] = i0 + e;
-          ++q;
-          atomicAdd(&h2[(w[e] >> kShift2) & (kBins2 - 1)], 1u);
-        }
-    }
-    n_cand += tot;
-  }
-  hc.flush(p.n_heads, heads);
+  HeadCounter hc(lo / p.n_c, p.n_c, p.n_heads, win, heads);
+  const uint32_t n_cand =
+      mask_pass(p.s, lo, hi, ub1, none, p.vec != 0, p.vec_keep != 0, p.keep, seg, hi - lo,
+                h2, tmp, [&](uint32_t f) { hc.add(f); });
+  hc.flush();
   __syncthreads();
   for (int i = threadIdx.x; i < kBins2; i += kThr)
     if (h2[i]) atomicAdd(g2 + i, h2[i]);
@@ -404,7 +508,7 @@ __global__ void __launch_bounds__(kThr)
     }
 
     // ---------------------------------------------------------- F: kept candidates
-    HeadCounter hf;
+    HeadCounter hf(lo / p.n_c, p.n_c, p.n_heads, win, heads);
     uint64_t ties_seen = 0;   // block-uniform: ties in earlier candidate tiles of this block
     for (uint32_t jb = 0; jb < n_cand; jb += kThr) {
       const uint32_t j = jb + threadIdx.x;
@@ -421,11 +525,16 @@ __global__ void __launch_bounds__(kThr)
       }
       if (kp && in_bounds(f >= lo && f < hi)) {
         p.keep[f] = 1;
-        hf.at(f, p.n_c, p.n_heads, heads);
-        ++hf.cnt;
+        hf.add(f);
       }
     }
-    hf.flush(p.n_heads, heads);
+    hf.flush();
+  }
+  __syncthreads();
+  {
+    const uint32_t h_lo = lo / p.n_c;   // the block's share of the per-head counts
+    for (int i = threadIdx.x; i < kHeadWin; i += kThr)
+      if (win[i] && in_bounds(h_lo + i < p.n_heads)) atomicAdd(heads + h_lo + i, win[i]);
   }
   if (!grid_barrier(sy, status, p.timeout_ns)) return;
 
@@ -453,7 +562,7 @@ __global__ void __launch_bounds__(kThr)
 // synchronisation only: histogram (read 1), bin of round 1, final mask bytes
 // and candidates in position order (read 2), rounds 2 and 3 and the tie ranks
 // on the candidates, then the kept candidates.  offsets[h] = h * k.
-__global__ void __launch_bounds__(kThr)
+__global__ void __launch_bounds__(kThr, 2)
     select_per_head_kernel(const float* __restrict__ s, uint32_t n_c, uint32_t n_heads,
                            uint32_t k, uint8_t* keep, int64_t* offsets, uint32_t* cand,
                            int vec, int vec_keep) {
@@ -465,7 +574,6 @@ __global__ void __launch_bounds__(kThr)
   const float* sh = s + lo;
   uint8_t* kh = keep + lo;
   uint32_t* seg = cand + lo;
-  const uint4* s4 = reinterpret_cast<const uint4*>(sh);
   const uint32_t* su = reinterpret_cast<const uint32_t*>(sh);
   const bool none = k == 0;
   // rows of this head start on 16 bytes only when n_c is a multiple of 4
@@ -481,17 +589,7 @@ __global__ void __launch_bounds__(kThr)
   if (!none) {
     for (int i = threadIdx.x; i < kBins1; i += kThr) h1[i] = 0;
     __syncthreads();
-    for (uint32_t i0 = 4 * threadIdx.x; i0 < n_c; i0 += kTile) {
-      if (v4 && i0 + 3 < n_c) {
-        const uint4 a = __ldg(s4 + i0 / 4);
-        atomicAdd(&h1[a.x >> kShift1], 1u);
-        atomicAdd(&h1[a.y >> kShift1], 1u);
-        atomicAdd(&h1[a.z >> kShift1], 1u);
-        atomicAdd(&h1[a.w >> kShift1], 1u);
-      } else {
-        for (uint32_t f = i0; f < i0 + 4 && f < n_c; ++f) atomicAdd(&h1[__ldg(su + f) >> kShift1], 1u);
-      }
-    }
+    hist_top(sh, 0, n_c, v4, h1);
     __syncthreads();
     uint64_t above;
     pick_bin<kBins1, true>(h1, k_rem, &b1, &above);
@@ -500,47 +598,8 @@ __global__ void __launch_bounds__(kThr)
   const uint32_t ub1 = static_cast<uint32_t>(b1);
   for (int i = threadIdx.x; i < kBins2; i += kThr) h2[i] = 0;
   __syncthreads();
-  uint32_t n_cand = 0;
-  for (uint32_t i0 = 4 * threadIdx.x, t0 = 0; t0 < n_c; i0 += kTile, t0 += kTile) {
-    uint32_t w[4] = {0, 0, 0, 0};
-    const bool full = i0 + 3 < n_c;
-    if (v4 && full) {
-      const uint4 a = __ldcs(s4 + i0 / 4);
-      w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-    } else {
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (i0 + e < n_c) w[e] = __ldcs(su + i0 + e);
-    }
-    uint32_t km = 0, cm = 0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint32_t d = w[e] >> kShift1;
-      const bool in = i0 + e < n_c;
-      km |= static_cast<uint32_t>(in && !none && d > ub1) << e;
-      cm |= static_cast<uint32_t>(in && !none && d == ub1) << e;
-    }
-    if (k4 && full) {
-      uint32_t word = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) word |= ((km >> e) & 1u) << (8 * e);
-      *reinterpret_cast<uint32_t*>(kh + i0) = word;
-    } else {
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (i0 + e < n_c) kh[i0 + e] = static_cast<uint8_t>((km >> e) & 1u);
-    }
-    uint32_t tot;
-    uint32_t q = n_cand + block_excl(__popc(cm), tmp, &tot);
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-      if ((cm >> e) & 1u) {
-        if (in_bounds(q < n_c)) seg[q] = i0 + e;
-        ++q;
-        atomicAdd(&h2[(w[e] >> kShift2) & (kBins2 - 1)], 1u);
-      }
-    n_cand += tot;
-  }
+  const uint32_t n_cand = mask_pass(sh, 0, n_c, ub1, none, v4, k4, kh, seg, n_c, h2, tmp,
+                                    [](uint32_t) {});
   __syncthreads();
   if (none) return;
   int b2;

@@ -407,34 +407,6 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   return p;
 }
 
-// a * b + c, rounded once, then clamped to [0, 1] (one FFMA with saturation).
-__device__ __forceinline__ float fma_sat(float a, float b, float c) {
-  float y;
-  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
-  return y;
-}
-
-// 2^x for x = kSatSpan * y - 125 with y in [0, 1] (so x in [-125, 126]): the
-// saturated input y is how callers clamp x on both sides in one instruction.
-// Same split and polynomial as exp2_poly2: j = shift + n with n = rint(x),
-// f = x - n in [-1/2, 1/2], 2^f by the degree-3 fit, n added to the exponent.
-// y's rounding adds at most kSatSpan * 2^-25 to x (relative 5e-6 on 2^x).
-constexpr float kSatSpan = 251.f;
-__device__ __forceinline__ float2 exp2_poly_sat2(float2 y) {
-  const float2 span = make_float2(kSatSpan, kSatSpan);
-  const float2 base = make_float2(12582787.f, 12582787.f);    // 1.5 * 2^23 - 125
-  const float2 j = ffma2(y, span, base);                       // 1.5 * 2^23 + n
-  const float2 t = fsub2(base, j);                             // -125 - n, exact
-  const float2 f = ffma2(y, span, t);                          // x - n
-  float2 p = ffma2(make_float2(0.05517177656292915f, 0.05517177656292915f), f,
-                   make_float2(0.2426113784313202f, 0.2426113784313202f));
-  p = ffma2(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
-  p = ffma2(p, f, make_float2(0.9999279975891113f, 0.9999279975891113f));
-  p.x = __int_as_float(imad_lo(__float_as_int(j.x), 1 << 23, __float_as_int(p.x)));
-  p.y = __int_as_float(imad_lo(__float_as_int(j.y), 1 << 23, __float_as_int(p.y)));
-  return p;
-}
-
 __device__ __forceinline__ float fmin3(float a, float b, float c) {
   float y;
   asm("min.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));

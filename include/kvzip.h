@@ -265,7 +265,8 @@ kvzip_status kvzip_select_noalloc(const float* scores, int64_t N, int64_t k, int
  *                           keep, offsets, ws)
  *
  * Every rank must run every step, in this order, with the same k.  Scores
- * 16-byte aligned, finite and >= 0; 1 <= N_local < 2^31.  All calls are
+ * 4-byte aligned (16-byte alignment is faster), finite and >= 0;
+ * 1 <= N_local < 2^31.  All calls are
  * asynchronous on `stream`; the caller orders its collectives after them.
  */
 int kvzip_select_shard_bins(int round);   /* 8192, 1024, 512; 0 for other rounds */

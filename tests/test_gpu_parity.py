@@ -260,13 +260,11 @@ def test_head_scores_bit_exact(kz, n_heads, n_c):
 def test_score_chunk_late_dominant_key(kz, jump):
     """A context key far down the sequence outscores every earlier key by `jump`
     in log2 units (all query rows share one direction, the key is a multiple of
-    it), far past the range of the pass-1 polynomial and of fp32 exponentials
-    taken against any earlier reference.  Pass 1 sums 2^(c s - m) against a
-    reference m fixed by the row's first chunk: a jump of 45 is summed as is,
-    70 pushes the sum past 2^64 (the reference moves up by 64), and 100 and
-    more send the chunk to the exact path (sum >= 2^100, the polynomial's
-    clamp at 2^126, or MUFU's inf).  Scores above 1e-30 match the oracle to
-    2e-3, the rest are below 1e-30."""
+    it), from well inside to far past the range of fp32 exponentials taken
+    against any earlier maximum (2^126 is the largest power of two the
+    polynomial exponentials reach, 2^128 overflows).  The online maximum must
+    rescale the row sum exactly.  Scores above 1e-30 match the oracle to 2e-3,
+    the rest are below 1e-30 (probabilities below 2^-126 flush to zero)."""
     B, G, n_in, n_c, d = 2, 2, 40, 2000, 128
     g = torch.Generator().manual_seed(int(jump))
     u = torch.randn(d, generator=g)
