@@ -63,6 +63,9 @@ def parse():
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-attention table")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the head-level / ablation kernel timings")
+    ap.add_argument("--only", choices=["select", "compact"], default=None,
+                    help="time one kernel alone on synthetic inputs of the workload's shape "
+                         "(a few hundred MB on the device; for profiling)")
     ap.add_argument("--dist-backend", choices=["nccl", "gloo"], default="nccl",
                     help="process-group backend under torchrun (gloo also runs several ranks "
                          "on one GPU, for testing the sharded path)")
@@ -196,10 +199,61 @@ def _resident_bytes(wl):
     return kv + wl.units * per_in * wl.d * 2 * (wl.G + 1)
 
 
+def run_only(args):
+    """One kernel alone: kvzip_select on L*H*n_c synthetic scores (skewed like
+    attention maxima), or kvzip_compact of one layer's K/V with a random keep
+    mask at ratio r.  Inputs exceed L2 (126 MB) at the 128K shape."""
+    from attention_score_reduction_b200 import kvzip as kz
+    dev = torch.device("cuda", 0)
+    wl = workload(args)
+    r = args.r if args.r is not None else wl.r[0]
+    peaks = bu.load_peaks(os.path.join(ROOT, "MEASURED_PEAKS.json"))
+    N = wl.units * wl.n_c
+    times = []
+    if args.only == "select":
+        s = synth.random_scores(wl.units, wl.n_c, seed=11, device=dev).reshape(-1)
+        k = kz.keep_count(r, N)
+        keep = torch.empty(N, dtype=torch.uint8, device=dev)
+        off = torch.empty(wl.units + 1, dtype=torch.int64, device=dev)
+        thr = torch.empty(1, dtype=torch.float32, device=dev)
+        ws = torch.zeros(kz.select_workspace_size(N, wl.units), dtype=torch.uint8, device=dev)
+        fn = lambda: kz.select(s, k, wl.units, keep, off, thr, ws)  # noqa: E731
+        nbytes = N * 4 + N
+    else:
+        units = wl.H      # one layer
+        k_c = torch.randn(units, wl.n_c, wl.d, device=dev).to(torch.bfloat16)
+        v = torch.randn_like(k_c)
+        s = synth.random_scores(units, wl.n_c, seed=12, device=dev).reshape(-1)
+        kept = kz.keep_count(r, s.numel())
+        keep, off, _ = kz.select(s, kept, units)
+        k_out = torch.empty(kept, wl.d, dtype=torch.bfloat16, device=dev)
+        v_out, pos = torch.empty_like(k_out), torch.empty(kept, dtype=torch.int32, device=dev)
+        fn = lambda: kz.compact(k_c, v, keep, off, kept, k_out, v_out, pos)  # noqa: E731
+        nbytes = s.numel() + kept * wl.d * 2 * 2 * 2 + kept * 4
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
+    for i in range(args.warmup + args.steps):
+        flush.fill_(i & 0xff)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            times.append(e0.elapsed_time(e1))
+    ms = sum(times) / len(times)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    print(json.dumps({"kernel": args.only, "workload": wl.name, "ms": ms, "bytes": nbytes,
+                      "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
+                      "peak_source": peaks["source"], "l2": "flushed before each launch"}))
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.only:
+        run_only(args)
         return
     rank, world, local = bu.dist_env()
     dev = torch.device("cuda", local % torch.cuda.device_count())
