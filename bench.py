@@ -336,7 +336,7 @@ def main():
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     launches = 0
-    with bu.ClockSampler(local) as clk:
+    with bu.ClockSampler(dev.index) as clk:
         start.record(stream)
         for _ in range(args.steps):
             launches += step(True)
