@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(256)
 }
 
 // Vector forms for n_c a multiple of 4 (every row then starts on 16 bytes).
-// head_max_v: two 16-byte loads in flight per thread.
+// head_max_v: four 16-byte loads in flight per thread.
 __global__ void __launch_bounds__(kHeadThreads)
     head_max_v(const float* __restrict__ s, int64_t n_c, int64_t segs, uint32_t* out) {
   const int64_t h = blockIdx.x / segs, sg = blockIdx.x % segs;
@@ -75,10 +75,13 @@ __global__ void __launch_bounds__(kHeadThreads)
   const int64_t n4 = (((j0 + kHeadSeg < n_c) ? j0 + kHeadSeg : n_c) - j0) / 4;
   const uint4* b4 = reinterpret_cast<const uint4*>(s + h * n_c + j0);
   uint32_t m = 0;
-  for (int64_t i = threadIdx.x; i < n4; i += 2 * kHeadThreads) {
-    const uint4 u0 = __ldcs(b4 + i);
-    const uint4 u1 = (i + kHeadThreads < n4) ? __ldcs(b4 + i + kHeadThreads) : make_uint4(0, 0, 0, 0);
-    m = max(m, max(max(max(u0.x, u0.y), max(u0.z, u0.w)), max(max(u1.x, u1.y), max(u1.z, u1.w))));
+  for (int64_t i = threadIdx.x; i < n4; i += 4 * kHeadThreads) {
+    uint4 u[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)   // zeros never raise a maximum of scores >= 0
+      u[q] = (i + q * kHeadThreads < n4) ? __ldcs(b4 + i + q * kHeadThreads) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) m = max(m, max(max(u[q].x, u[q].y), max(u[q].z, u[q].w)));
   }
   m = __reduce_max_sync(0xffffffffu, m);
   __shared__ uint32_t red[kHeadThreads / 32];
