@@ -56,8 +56,10 @@ constexpr int kShift1 = 19, kShift2 = 9;  // digit of round 1: bits 31..19, roun
 // Workspace layout (bytes).  [kOffSync, zero_end) is zeroed by the host before
 // every launch; the rest is written before it is read.
 constexpr size_t kOffStatus = 0;          // sticky status word (kvzip_workspace_status)
-constexpr size_t kOffSync = 256;          // barrier count, generation, abort flag
-constexpr size_t kOffH1 = 512;
+constexpr size_t kOffSync = 256;          // grid-barrier counters (Sync), zeroed per launch
+constexpr int kBarGroups = 16;            // first-level barrier counters
+constexpr size_t kLine = 128;             // one counter per 128-byte line
+constexpr size_t kOffH1 = kOffSync + (kBarGroups + 2) * kLine;
 constexpr size_t kOffH2 = kOffH1 + kBins1 * 4;
 constexpr size_t kOffH3 = kOffH2 + kBins2 * 4;
 constexpr size_t kOffHeads = kOffH3 + kBins3 * 4;
@@ -98,8 +100,15 @@ struct Params {
   int test_stall;        // test hook: block 0 never reaches a barrier, so the others time out
 };
 
+// Grid-barrier words, each on its own 128-byte line: kBarGroups first-level
+// arrival counters, the second-level counter, then the generation and abort
+// flag.  Arrivals on one address serialise in L2 (and cross between the two
+// dies for half of the SMs), so the blocks first arrive in kBarGroups groups
+// (block b in group b % kBarGroups) and only each group's last block arrives
+// on the second level.
 struct Sync {
-  unsigned int count;
+  unsigned int group[kBarGroups][kLine / 4];
+  unsigned int top[kLine / 4];
   unsigned int gen;
   unsigned int abort;
 };
@@ -115,8 +124,17 @@ __device__ bool grid_barrier(Sync* sy, uint32_t* status, uint64_t timeout_ns) {
     const unsigned int g = *vgen;
     __threadfence();
     int ok = 1;
-    if (atomicAdd(&sy->count, 1u) == gridDim.x - 1) {
-      atomicExch(&sy->count, 0u);
+    const unsigned int n_groups = min(gridDim.x, static_cast<unsigned int>(kBarGroups));
+    const unsigned int grp = blockIdx.x % n_groups;
+    const unsigned int grp_size = (gridDim.x - grp + n_groups - 1) / n_groups;
+    bool last = false;
+    if (atomicAdd(&sy->group[grp][0], 1u) == grp_size - 1) {
+      atomicExch(&sy->group[grp][0], 0u);
+      __threadfence();
+      last = atomicAdd(&sy->top[0], 1u) == n_groups - 1;
+    }
+    if (last) {
+      atomicExch(&sy->top[0], 0u);
       __threadfence();
       atomicAdd(&sy->gen, 1u);
     } else {
