@@ -135,7 +135,8 @@ def compress_from_host(comp: Compressor, k_ctx_h, v_h, q_chunks_h, ks_chunks_h, 
     reusable device tensors: "k_ctx", "v", and lists "q", "ks" of chunk buffers.
     When the lists are shorter than the chunk list they are used as a ring:
     chunk c goes into buffer c % len, and its upload waits until the scorer has
-    finished the chunk that last used that buffer.  ``host_out`` (pinned)
+    finished the chunk that last used that buffer.  V is uploaded after the first
+    chunk's inputs, under the scoring; only compaction waits for it.  ``host_out`` (pinned)
     receives "k", "v", "pos", "offsets".  Uploads run on a side stream, each
     chunk's upload recorded by an event the scorer waits on.
     Returns (Compressed on the device, host_out, bytes_h2d, bytes_d2h).
@@ -149,12 +150,11 @@ def compress_from_host(comp: Compressor, k_ctx_h, v_h, q_chunks_h, ks_chunks_h, 
     h2d = 0
     with torch.cuda.stream(copy):
         dev_bufs["k_ctx"].copy_(k_ctx_h, non_blocking=True)
-        dev_bufs["v"].copy_(v_h, non_blocking=True)
-        h2d += k_ctx_h.numel() * k_ctx_h.element_size() + v_h.numel() * v_h.element_size()
-        ev_kv = torch.cuda.Event()
-        ev_kv.record(copy)
+        h2d += k_ctx_h.numel() * k_ctx_h.element_size()
+        ev_k = torch.cuda.Event()
+        ev_k.record(copy)
     comp.reset()
-    main.wait_event(ev_kv)
+    main.wait_event(ev_k)           # scoring needs the keys; V only at compaction
     freed = [None] * n_buf          # event: the scorer is done with this ring slot
     for c, (qh, ksh) in enumerate(zip(q_chunks_h, ks_chunks_h)):
         slot = c % n_buf
@@ -175,6 +175,19 @@ def compress_from_host(comp: Compressor, k_ctx_h, v_h, q_chunks_h, ks_chunks_h, 
         done = torch.cuda.Event()
         done.record(main)
         freed[slot] = done
+        if c == 0:                  # V rides behind the first chunk, under the scoring
+            with torch.cuda.stream(copy):
+                dev_bufs["v"].copy_(v_h, non_blocking=True)
+                h2d += v_h.numel() * v_h.element_size()
+                ev_v = torch.cuda.Event()
+                ev_v.record(copy)
+    if not q_chunks_h:
+        with torch.cuda.stream(copy):
+            dev_bufs["v"].copy_(v_h, non_blocking=True)
+            h2d += v_h.numel() * v_h.element_size()
+            ev_v = torch.cuda.Event()
+            ev_v.record(copy)
+    main.wait_event(ev_v)
     kept = comp.select(r)
     if comp.group is not None:    # this rank's share of the global count (one small read)
         kept = int(comp.offsets[-1])
