@@ -266,75 +266,73 @@ __device__ uint32_t mask_pass(const float* __restrict__ s, uint32_t lo, uint32_t
   const uint32_t* su = reinterpret_cast<const uint32_t*>(s);
   uint32_t n_cand = 0;   // block-uniform
   for (uint32_t g0 = lo; g0 < hi; g0 += 4 * kTile) {
-    uint32_t w[4][4];
-    uint32_t i0[4];
-    bool full[4];
+    const uint32_t ib = g0 + 4 * threadIdx.x;   // this thread's first score of tile 0
+    uint4 a[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      i0[q] = g0 + q * kTile + 4 * threadIdx.x;
-      full[q] = i0[q] + 3 < hi;
-      if (vec && full[q]) {
-        const uint4 a = __ldcs(s4 + i0[q] / 4);
-        w[q][0] = a.x;
-        w[q][1] = a.y;
-        w[q][2] = a.z;
-        w[q][3] = a.w;
+    for (int q = 0; q < 4; ++q) {               // four loads in flight
+      const uint32_t i0 = ib + q * kTile;
+      if (vec && i0 + 3 < hi) {
+        a[q] = __ldcs(s4 + i0 / 4);
       } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) w[q][e] = (i0[q] + e < hi) ? __ldcs(su + i0[q] + e) : 0u;
+        a[q].x = (i0 + 0 < hi) ? __ldcs(su + i0 + 0) : 0u;
+        a[q].y = (i0 + 1 < hi) ? __ldcs(su + i0 + 1) : 0u;
+        a[q].z = (i0 + 2 < hi) ? __ldcs(su + i0 + 2) : 0u;
+        a[q].w = (i0 + 3 < hi) ? __ldcs(su + i0 + 3) : 0u;
       }
     }
-    uint32_t km[4], cm[4];
+    // classify tile by tile; only the candidate bits stay live across the scan
+    uint32_t cm = 0;   // bit 4q + e: score e of tile q is a candidate
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      km[q] = cm[q] = 0;
+      const uint32_t i0 = ib + q * kTile;
+      const uint32_t w[4] = {a[q].x, a[q].y, a[q].z, a[q].w};
+      uint32_t km = 0, word = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const uint32_t d = w[q][e] >> kShift1;
-        const bool in = i0[q] + e < hi && !none;
-        km[q] |= static_cast<uint32_t>(in && d > b1) << e;
-        cm[q] |= static_cast<uint32_t>(in && d == b1) << e;
+        const uint32_t d = w[e] >> kShift1;
+        const bool in = i0 + e < hi && !none;
+        const bool k1 = in && d > b1, c1 = in && d == b1;
+        km |= static_cast<uint32_t>(k1) << e;
+        word |= static_cast<uint32_t>(k1) << (8 * e);
+        if (c1) {
+          cm |= 1u << (4 * q + e);
+          atomicAdd(&h2[(w[e] >> kShift2) & (kBins2 - 1)], 1u);
+        }
       }
-      if (vec_keep && full[q]) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) word |= ((km[q] >> e) & 1u) << (8 * e);
-        *reinterpret_cast<uint32_t*>(keep + i0[q]) = word;
+      if (vec_keep && i0 + 3 < hi) {
+        *reinterpret_cast<uint32_t*>(keep + i0) = word;   // 0 for candidates, set later
       } else {
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          if (i0[q] + e < hi) keep[i0[q] + e] = static_cast<uint8_t>((km[q] >> e) & 1u);
+          if (i0 + e < hi) keep[i0 + e] = static_cast<uint8_t>((km >> e) & 1u);
       }
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        if ((km[q] >> e) & 1u) on_kept(i0[q] + e);
+        if ((km >> e) & 1u) on_kept(i0 + e);
     }
     // candidate positions: counts of tiles 0/1 and 2/3 packed in 16-bit halves
     // (a tile has at most kTile = 2048 candidates, so the halves never carry)
+    const uint32_t c0 = __popc(cm & 0xFu), c1 = __popc(cm & 0xF0u), c2 = __popc(cm & 0xF00u),
+                   c3 = __popc(cm & 0xF000u);
     uint32_t ex01, ex23, t01, t23;
-    block_excl2(__popc(cm[0]) | (__popc(cm[1]) << 16), __popc(cm[2]) | (__popc(cm[3]) << 16),
-                tmp, &ex01, &ex23, &t01, &t23);
-    uint32_t base[4], pos[4];
-    base[0] = n_cand;
-    base[1] = base[0] + (t01 & 0xFFFFu);
-    base[2] = base[1] + (t01 >> 16);
-    base[3] = base[2] + (t23 & 0xFFFFu);
-    pos[0] = base[0] + (ex01 & 0xFFFFu);
-    pos[1] = base[1] + (ex01 >> 16);
-    pos[2] = base[2] + (ex23 & 0xFFFFu);
-    pos[3] = base[3] + (ex23 >> 16);
+    block_excl2(c0 | (c1 << 16), c2 | (c3 << 16), tmp, &ex01, &ex23, &t01, &t23);
+    if (cm) {
+      const uint32_t b0 = n_cand, bq1 = b0 + (t01 & 0xFFFFu), bq2 = bq1 + (t01 >> 16),
+                     bq3 = bq2 + (t23 & 0xFFFFu);
+      const uint32_t pos[4] = {b0 + (ex01 & 0xFFFFu), bq1 + (ex01 >> 16), bq2 + (ex23 & 0xFFFFu),
+                               bq3 + (ex23 >> 16)};
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      uint32_t x = pos[q];
+      for (int q = 0; q < 4; ++q) {
+        uint32_t x = pos[q];
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if ((cm[q] >> e) & 1u) {
-          if (in_bounds(x < seg_cap)) seg[x] = i0[q] + e;
-          ++x;
-          atomicAdd(&h2[(w[q][e] >> kShift2) & (kBins2 - 1)], 1u);
-        }
+        for (int e = 0; e < 4; ++e)
+          if ((cm >> (4 * q + e)) & 1u) {
+            if (in_bounds(x < seg_cap)) seg[x] = ib + q * kTile + e;
+            ++x;
+          }
+      }
     }
-    n_cand = base[3] + (t23 >> 16);
+    n_cand += (t01 & 0xFFFFu) + (t01 >> 16) + (t23 & 0xFFFFu) + (t23 >> 16);
   }
   return n_cand;
 }
@@ -512,38 +510,44 @@ __global__ void __launch_bounds__(kThr, 2)
     take_eq = k_rem;                                   // scores equal to tau that are kept
     const uint64_t n_eq = __ldcg(g3 + b3);
     rank_ties = take_eq < n_eq;                        // the same decision in every block
-    if (rank_ties) {
+    HeadCounter hf(lo / p.n_c, p.n_c, p.n_heads, win, heads);
+    if (!rank_ties) {
+      // ---------------------------------------------------------- F: kept candidates
+      for (uint32_t j = threadIdx.x; j < n_cand; j += kThr) {
+        const uint32_t f = seg[j];
+        if (__ldg(su + f) >= tau && in_bounds(f >= lo && f < hi)) {
+          p.keep[f] = 1;
+          hf.add(f);
+        }
+      }
+    } else {
+      // Ties straddle the threshold: rank them in flat order.  Each thread takes a
+      // contiguous run of the block's candidates (which are in flat order), so one
+      // block scan of per-thread tie counts and one scan over the blocks give
+      // every tie its global rank.
+      const uint32_t run = (n_cand + kThr - 1) / kThr;
+      const uint32_t j0 = min(threadIdx.x * run, n_cand), j1 = min(j0 + run, n_cand);
       uint32_t c = 0;
-      for (uint32_t j = threadIdx.x; j < n_cand; j += kThr) c += (__ldg(su + seg[j]) == tau);
+      for (uint32_t j = j0; j < j1; ++j) c += (__ldg(su + seg[j]) == tau);
       uint32_t tot;
-      block_excl(c, tmp, &tot);
+      const uint32_t mine_before = block_excl(c, tmp, &tot);
       if (threadIdx.x == 0) blk_tie[blockIdx.x] = tot;
       if (!grid_barrier(sy, status, p.timeout_ns)) return;
       uint32_t part = 0;
       for (uint32_t b = threadIdx.x; b < blockIdx.x; b += kThr) part += __ldcg(blk_tie + b);
       block_excl(part, tmp, &tot);
       tie_base = tot;
-    }
-
-    // ---------------------------------------------------------- F: kept candidates
-    HeadCounter hf(lo / p.n_c, p.n_c, p.n_heads, win, heads);
-    uint64_t ties_seen = 0;   // block-uniform: ties in earlier candidate tiles of this block
-    for (uint32_t jb = 0; jb < n_cand; jb += kThr) {
-      const uint32_t j = jb + threadIdx.x;
-      const bool in = j < n_cand;
-      const uint32_t f = in ? seg[j] : 0u;
-      const uint32_t w = in ? __ldg(su + f) : 0u;
-      const bool eq = in && w == tau;
-      bool kp = in && (w > tau || (eq && !rank_ties));
-      if (rank_ties) {
-        uint32_t tot;
-        const uint32_t r = block_excl(eq ? 1u : 0u, tmp, &tot);
-        kp = kp || (eq && tie_base + ties_seen + r < take_eq);
-        ties_seen += tot;
-      }
-      if (kp && in_bounds(f >= lo && f < hi)) {
-        p.keep[f] = 1;
-        hf.add(f);
+      // ---------------------------------------------------------- F: kept candidates
+      uint64_t rank = tie_base + mine_before;
+      for (uint32_t j = j0; j < j1; ++j) {
+        const uint32_t f = seg[j];
+        const uint32_t w = __ldg(su + f);
+        bool kp = w > tau;
+        if (w == tau) kp = rank++ < take_eq;
+        if (kp && in_bounds(f >= lo && f < hi)) {
+          p.keep[f] = 1;
+          hf.add(f);
+        }
       }
     }
     hf.flush();
@@ -639,20 +643,26 @@ __global__ void __launch_bounds__(kThr, 2)
   const uint32_t tau = pre2 | static_cast<uint32_t>(b3);
   const uint64_t take_eq = k_rem;
   const bool rank_ties = take_eq < h3[b3];
-  uint64_t ties_seen = 0;
-  for (uint32_t jb = 0; jb < n_cand; jb += kThr) {
-    const uint32_t j = jb + threadIdx.x;
-    const bool in = j < n_cand;
-    const uint32_t f = in ? seg[j] : 0u;
-    const uint32_t w = in ? __ldg(su + f) : 0u;
-    const bool eq = in && w == tau;
-    bool kp = in && (w > tau || (eq && !rank_ties));
-    if (rank_ties) {
-      uint32_t tot;
-      const uint32_t r = block_excl(eq ? 1u : 0u, tmp, &tot);
-      kp = kp || (eq && ties_seen + r < take_eq);
-      ties_seen += tot;
+  if (!rank_ties) {
+    for (uint32_t j = threadIdx.x; j < n_cand; j += kThr) {
+      const uint32_t f = seg[j];
+      if (__ldg(su + f) >= tau && in_bounds(f < n_c)) kh[f] = 1;
     }
+    return;
+  }
+  // ties straddle the threshold: contiguous runs of candidates per thread, one
+  // block scan of the per-thread tie counts gives each tie its rank in position order
+  const uint32_t run = (n_cand + kThr - 1) / kThr;
+  const uint32_t j0 = min(threadIdx.x * run, n_cand), j1 = min(j0 + run, n_cand);
+  uint32_t c = 0;
+  for (uint32_t j = j0; j < j1; ++j) c += (__ldg(su + seg[j]) == tau);
+  uint32_t tot;
+  uint64_t rank = block_excl(c, tmp, &tot);
+  for (uint32_t j = j0; j < j1; ++j) {
+    const uint32_t f = seg[j];
+    const uint32_t w = __ldg(su + f);
+    bool kp = w > tau;
+    if (w == tau) kp = rank++ < take_eq;
     if (kp && in_bounds(f < n_c)) kh[f] = 1;
   }
 }
