@@ -10,16 +10,19 @@
 //   B  every block finds, from the merged histogram, the bin b1 that holds the
 //      k-th largest score (the same answer in every block).
 //   C  every block reads its range again (read 2) and writes the final mask
-//      byte of every score outside bin b1 (kept iff its bin is above b1).  The
-//      flat indices of the scores inside bin b1 (the candidates) are appended,
-//      in flat order, to the block's own segment of a candidate buffer, and
-//      their next 10 bits are histogrammed; grid barrier.
+//      byte of every score outside bin b1 (kept iff its bin is above b1).  Each
+//      warp owns a contiguous slice of the block's range and appends the
+//      scores inside bin b1 (the candidates), as (flat index, score bits)
+//      pairs in flat order, to its own segment of a candidate buffer, placed
+//      by a warp scan (no block barrier in the streaming loop); their next 10
+//      bits are histogrammed; grid barrier.
 //   D  bin b2 of round 2, then a histogram of the last 9 bits over the
-//      candidates that match b1 b2 (gathered by index); grid barrier.
+//      candidates that match b1 b2 (coalesced reads of the pairs); each block
+//      also stores its own round-3 histogram; grid barrier.
 //   E  bin b3 gives the threshold tau exactly.  If fewer scores equal to tau
-//      are kept than exist, every block counts its candidates equal to tau and,
-//      after a barrier, sums the counts of the blocks before it: the flat-order
-//      rank of its first tie.
+//      are kept than exist, the ties are ranked in flat order: the blocks'
+//      stored histograms give the ties before this block, a per-warp count
+//      the ties before this warp, and a ballot walk the rest.
 //   F  every block sets the mask of its kept candidates; grid barrier.
 //   G  block 0 turns the per-head kept counts into offsets and writes tau.
 //
@@ -48,7 +51,9 @@ namespace kvzip {
 namespace {
 
 constexpr int kThr = 512;                // threads per block
+constexpr int kWarps = kThr / 32;
 constexpr int kTile = kThr * 4;          // scores per block tile (4 per thread, 16-byte loads)
+constexpr int kWarpStep = 4 * 128;       // scores per warp step of the mask pass (4 loads of 512 B)
 constexpr int kMaxBlocks = 1024;
 constexpr int kBins1 = 8192, kBins2 = 1024, kBins3 = 512;
 constexpr int kShift1 = 19, kShift2 = 9;  // digit of round 1: bits 31..19, round 2: 18..9, round 3: 8..0
@@ -68,19 +73,26 @@ __host__ __device__ size_t up256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct Layout {
   size_t zero_end;    // end of the region zeroed before each launch
-  size_t off_blk;     // blk_cand[kMaxBlocks], blk_tie[kMaxBlocks]
-  size_t off_cand;    // candidate flat indices, one segment per block
+  size_t off_h3blk;   // every block's round-3 histogram [blocks][kBins3]
+  size_t off_cand;    // candidate (flat index, score bits) pairs
   size_t total;
 };
 
-// Candidate capacity: every block's segment holds its whole range (ranges are
-// multiples of 4 scores), so the buffer never overflows.
+// The most blocks a launch over N scores uses (no block gets less than a tile).
+__host__ __device__ int64_t max_blocks(int64_t N) {
+  const int64_t b = (N + kTile - 1) / kTile;
+  return b < 1 ? 1 : (b > kMaxBlocks ? kMaxBlocks : b);
+}
+
+// Candidate capacity: the pair of score f lives at cand[f] at most (a warp's
+// segment starts at its slice's first flat index and holds the whole slice),
+// so the buffer never overflows.
 __host__ __device__ Layout layout(int64_t N, int64_t n_heads) {
   Layout L;
   L.zero_end = up256(kOffHeads + static_cast<size_t>(n_heads) * 4);
-  L.off_blk = L.zero_end;
-  L.off_cand = L.off_blk + up256(2 * kMaxBlocks * 4);
-  L.total = L.off_cand + up256((static_cast<size_t>(N) + 4 * kMaxBlocks) * 4);
+  L.off_h3blk = L.zero_end;
+  L.off_cand = L.off_h3blk + up256(static_cast<size_t>(max_blocks(N)) * kBins3 * 4);
+  L.total = L.off_cand + up256(static_cast<size_t>(N) * 8);
   return L;
 }
 
@@ -92,8 +104,8 @@ struct Params {
   int64_t* offsets;
   float* threshold;
   uint8_t* ws;
-  uint32_t* cand;        // base of the candidate buffer
-  uint32_t seg;          // scores per block range (multiple of 4)
+  uint2* cand;           // base of the candidate buffer
+  uint32_t seg;          // scores per block range (multiple of 128)
   uint64_t timeout_ns;
   int vec;               // scores 16-byte aligned: 16-byte loads
   int vec_keep;          // keep 4-byte aligned: 4-byte mask stores
@@ -184,42 +196,6 @@ __device__ __forceinline__ uint32_t block_excl(uint32_t v, uint32_t* tmp, uint32
   return before + inc - v;
 }
 
-// The same for two words per thread in one pass (one pair of barriers).
-__device__ __forceinline__ void block_excl2(uint32_t v0, uint32_t v1, uint32_t* tmp,
-                                            uint32_t* ex0, uint32_t* ex1, uint32_t* tot0,
-                                            uint32_t* tot1) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t a = v0, b = v1;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t na = __shfl_up_sync(0xffffffffu, a, o);
-    const uint32_t nb = __shfl_up_sync(0xffffffffu, b, o);
-    if (lane >= o) {
-      a += na;
-      b += nb;
-    }
-  }
-  if (lane == 31) {
-    tmp[warp] = a;
-    tmp[kThr / 32 + warp] = b;
-  }
-  __syncthreads();
-  uint32_t ba = 0, bb = 0, ta = 0, tb = 0;
-#pragma unroll
-  for (int w = 0; w < kThr / 32; ++w) {
-    const uint32_t xa = tmp[w], xb = tmp[kThr / 32 + w];
-    ba += (w < warp) ? xa : 0u;
-    bb += (w < warp) ? xb : 0u;
-    ta += xa;
-    tb += xb;
-  }
-  __syncthreads();
-  *ex0 = ba + a - v0;
-  *ex1 = bb + b - v1;
-  *tot0 = ta;
-  *tot1 = tb;
-}
-
 // Round-1 histogram of the top 13 bits of the scores [lo, hi) of s (indices
 // relative to s) into shared memory: four 16-byte loads in flight per thread.
 __device__ __forceinline__ void hist_top(const float* __restrict__ s, uint32_t lo, uint32_t hi,
@@ -251,90 +227,118 @@ __device__ __forceinline__ void hist_top(const float* __restrict__ s, uint32_t l
   }
 }
 
-// Second pass over the scores [lo, hi) of s, four tiles of kTile per step
-// (four 16-byte loads in flight per thread): the final mask byte of every
-// score outside bin b1 (kept iff its bin is above b1; 0 for candidates, set
-// later), the candidates' indices appended to seg in index order (positions
-// from one block scan of packed per-tile counts), their round-2 digits
-// histogrammed into h2, and on_kept(f) for every kept score (in increasing f
-// per thread).  Indices are relative to s; returns the block's candidate count.
-template <class OnKept>
-__device__ uint32_t mask_pass(const float* __restrict__ s, uint32_t lo, uint32_t hi, uint32_t b1,
-                              bool none, bool vec, bool vec_keep, uint8_t* keep, uint32_t* seg,
-                              uint32_t seg_cap, uint32_t* h2, uint32_t* tmp, OnKept on_kept) {
+// A warp's slice of the block range [lo, hi): 16 slices of equal length, each
+// a multiple of 32 scores (so slices start on 16 bytes when lo does).
+__device__ __forceinline__ void warp_slice(uint32_t lo, uint32_t hi, uint32_t* wl, uint32_t* wh) {
+  const uint32_t len = ((hi - lo + kWarps - 1) / kWarps + 31) & ~31u;
+  *wl = min(lo + (threadIdx.x >> 5) * len, hi);
+  *wh = min(*wl + len, hi);
+}
+
+// Round-1 decision per score, from its bits w (scores >= 0 order like their
+// bits): kept iff w > lim (its 13-bit bin is above b1); a candidate iff
+// w - base < width (its bin is b1).  With k = 0 nothing is kept or a candidate.
+struct Round1 {
+  uint32_t lim, base, width;
+  __device__ Round1(int b1, bool none) {
+    const uint32_t b = static_cast<uint32_t>(b1);
+    lim = none ? 0xFFFFFFFFu : ((b << kShift1) | ((1u << kShift1) - 1));
+    base = none ? 0u : (b << kShift1);
+    width = none ? 0u : (1u << kShift1);
+  }
+};
+
+// Second pass over a warp's slice [wl, wh) of s, 512 scores per step (four
+// 16-byte loads in flight per lane): the final mask byte of every score
+// outside bin b1 (0 for candidates, set later), the candidates appended as
+// (flat index, bits) pairs to seg in flat order (positions from one warp scan
+// of per-load counts packed in bytes), their round-2 digits histogrammed into
+// h2, and cnt.add4(i, km) for each group of four scores at i with kept bits
+// km (in increasing i per lane).  Returns the warp's candidate count.
+template <class Counter>
+__device__ uint32_t mask_pass(const float* __restrict__ s, uint32_t wl, uint32_t wh,
+                              const Round1 r1, bool vec, bool vec_keep, uint8_t* keep,
+                              uint2* seg, uint32_t* h2, Counter& cnt) {
   const uint4* s4 = reinterpret_cast<const uint4*>(s);
   const uint32_t* su = reinterpret_cast<const uint32_t*>(s);
-  uint32_t n_cand = 0;   // block-uniform
-  for (uint32_t g0 = lo; g0 < hi; g0 += 4 * kTile) {
-    const uint32_t ib = g0 + 4 * threadIdx.x;   // this thread's first score of tile 0
+  const uint32_t lane = threadIdx.x & 31;
+  uint32_t n_w = 0;   // warp-uniform
+  for (uint32_t g0 = wl; g0 < wh; g0 += kWarpStep) {
+    const uint32_t ib = g0 + 4 * lane;   // this lane's first score of load 0
     uint4 a[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {               // four loads in flight
-      const uint32_t i0 = ib + q * kTile;
-      if (vec && i0 + 3 < hi) {
+    for (int q = 0; q < 4; ++q) {        // four loads in flight
+      const uint32_t i0 = ib + q * 128;
+      if (vec && i0 + 3 < wh) {
         a[q] = __ldcs(s4 + i0 / 4);
       } else {
-        a[q].x = (i0 + 0 < hi) ? __ldcs(su + i0 + 0) : 0u;
-        a[q].y = (i0 + 1 < hi) ? __ldcs(su + i0 + 1) : 0u;
-        a[q].z = (i0 + 2 < hi) ? __ldcs(su + i0 + 2) : 0u;
-        a[q].w = (i0 + 3 < hi) ? __ldcs(su + i0 + 3) : 0u;
+        a[q].x = (i0 + 0 < wh) ? __ldcs(su + i0 + 0) : 0u;
+        a[q].y = (i0 + 1 < wh) ? __ldcs(su + i0 + 1) : 0u;
+        a[q].z = (i0 + 2 < wh) ? __ldcs(su + i0 + 2) : 0u;
+        a[q].w = (i0 + 3 < wh) ? __ldcs(su + i0 + 3) : 0u;
       }
     }
-    // classify tile by tile; only the candidate bits stay live across the scan
-    uint32_t cm = 0;   // bit 4q + e: score e of tile q is a candidate
+    uint32_t cm = 0, packed = 0;   // candidate bits (4q + e); candidates per load, one byte each
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const uint32_t i0 = ib + q * kTile;
+      const uint32_t i0 = ib + q * 128;
       const uint32_t w[4] = {a[q].x, a[q].y, a[q].z, a[q].w};
-      uint32_t km = 0, word = 0;
+      const uint32_t n_in = i0 < wh ? min(wh - i0, 4u) : 0u;
+      const uint32_t vm = (1u << n_in) - 1u;
+      uint32_t km = 0, cq = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const uint32_t d = w[e] >> kShift1;
-        const bool in = i0 + e < hi && !none;
-        const bool k1 = in && d > b1, c1 = in && d == b1;
-        km |= static_cast<uint32_t>(k1) << e;
-        word |= static_cast<uint32_t>(k1) << (8 * e);
-        if (c1) {
-          cm |= 1u << (4 * q + e);
-          atomicAdd(&h2[(w[e] >> kShift2) & (kBins2 - 1)], 1u);
-        }
+        km |= static_cast<uint32_t>(w[e] > r1.lim) << e;
+        cq |= static_cast<uint32_t>(w[e] - r1.base < r1.width) << e;
       }
-      if (vec_keep && i0 + 3 < hi) {
-        *reinterpret_cast<uint32_t*>(keep + i0) = word;   // 0 for candidates, set later
+      km &= vm;
+      cq &= vm;
+      if (vec_keep && n_in == 4) {
+        // bit e of km to bit 8e (the shifted copies of km do not overlap, so no carries)
+        *reinterpret_cast<uint32_t*>(keep + i0) = (km * 0x00204081u) & 0x01010101u;
       } else {
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          if (i0 + e < hi) keep[i0 + e] = static_cast<uint8_t>((km >> e) & 1u);
+          if (e < static_cast<int>(n_in)) keep[i0 + e] = static_cast<uint8_t>((km >> e) & 1u);
       }
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if ((km >> e) & 1u) on_kept(i0 + e);
-    }
-    // candidate positions: counts of tiles 0/1 and 2/3 packed in 16-bit halves
-    // (a tile has at most kTile = 2048 candidates, so the halves never carry)
-    const uint32_t c0 = __popc(cm & 0xFu), c1 = __popc(cm & 0xF0u), c2 = __popc(cm & 0xF00u),
-                   c3 = __popc(cm & 0xF000u);
-    uint32_t ex01, ex23, t01, t23;
-    block_excl2(c0 | (c1 << 16), c2 | (c3 << 16), tmp, &ex01, &ex23, &t01, &t23);
-    if (cm) {
-      const uint32_t b0 = n_cand, bq1 = b0 + (t01 & 0xFFFFu), bq2 = bq1 + (t01 >> 16),
-                     bq3 = bq2 + (t23 & 0xFFFFu);
-      const uint32_t pos[4] = {b0 + (ex01 & 0xFFFFu), bq1 + (ex01 >> 16), bq2 + (ex23 & 0xFFFFu),
-                               bq3 + (ex23 >> 16)};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t x = pos[q];
+      if (cq) {
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          if ((cm >> (4 * q + e)) & 1u) {
-            if (in_bounds(x < seg_cap)) seg[x] = ib + q * kTile + e;
-            ++x;
-          }
+          if ((cq >> e) & 1u) atomicAdd(&h2[(w[e] >> kShift2) & (kBins2 - 1)], 1u);
       }
+      cnt.add4(i0, km);
+      cm |= cq << (4 * q);
+      packed |= static_cast<uint32_t>(__popc(cq)) << (8 * q);
     }
-    n_cand += (t01 & 0xFFFFu) + (t01 >> 16) + (t23 & 0xFFFFu) + (t23 >> 16);
+    if (__any_sync(0xffffffffu, cm != 0)) {
+      // per-load counts are <= 128 per warp, so the byte lanes of the scan never carry
+      uint32_t inc = packed;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t n = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= static_cast<uint32_t>(o)) inc += n;
+      }
+      const uint32_t tot = __shfl_sync(0xffffffffu, inc, 31), ex = inc - packed;
+      const uint32_t t0 = tot & 0xFFu, t1 = (tot >> 8) & 0xFFu, t2 = (tot >> 16) & 0xFFu,
+                     t3 = tot >> 24;
+      if (cm) {
+        const uint32_t before[4] = {0u, t0, t0 + t1, t0 + t1 + t2};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t x = n_w + before[q] + ((ex >> (8 * q)) & 0xFFu);
+          const uint32_t w[4] = {a[q].x, a[q].y, a[q].z, a[q].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if ((cm >> (4 * q + e)) & 1u) {
+              if (in_bounds(x < wh - wl)) seg[x] = make_uint2(ib + q * 128 + e, w[e]);
+              ++x;
+            }
+        }
+      }
+      n_w += t0 + t1 + t2 + t3;
+    }
   }
-  return n_cand;
+  return n_w;
 }
 
 // The bin (scanning from the top) that holds the k_rem-th largest element of a
@@ -409,6 +413,17 @@ struct HeadCounter {
     }
     ++cnt;
   }
+  // The kept ones (bits of km) among the four scores i..i+3.
+  __device__ __forceinline__ void add4(uint32_t i, uint32_t km) {
+    if (!km) return;
+    if (i + 3 < end) {   // all four in the current head (indices only grow)
+      cnt += __popc(km);
+      return;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if ((km >> e) & 1u) add(i + e);
+  }
   __device__ __forceinline__ void flush() {
     if (!cnt) return;
     if (h - h_lo < static_cast<uint32_t>(kHeadWin))
@@ -419,12 +434,17 @@ struct HeadCounter {
   }
 };
 
+struct NoCounter {
+  __device__ __forceinline__ void add4(uint32_t, uint32_t) {}
+};
+
 __global__ void __launch_bounds__(kThr, 2)
     select_fused_kernel(const Params p) {
   __shared__ uint32_t h1[kBins1];       // round-1 histogram (32 KB), reused by later rounds
   __shared__ uint32_t h2[kBins2];
   __shared__ uint32_t tmp[2 * (kThr / 32)];
   __shared__ uint32_t win[kHeadWin];
+  __shared__ uint32_t wtie[kWarps];
 
   uint32_t* status = reinterpret_cast<uint32_t*>(p.ws + kOffStatus);
   Sync* sy = reinterpret_cast<Sync*>(p.ws + kOffSync);
@@ -433,13 +453,14 @@ __global__ void __launch_bounds__(kThr, 2)
   uint32_t* g3 = reinterpret_cast<uint32_t*>(p.ws + kOffH3);
   uint32_t* heads = reinterpret_cast<uint32_t*>(p.ws + kOffHeads);
   const Layout Lw = layout(p.N, p.n_heads);
-  uint32_t* blk_cand = reinterpret_cast<uint32_t*>(p.ws + Lw.off_blk);
-  uint32_t* blk_tie = blk_cand + kMaxBlocks;
+  uint32_t* h3blk = reinterpret_cast<uint32_t*>(p.ws + Lw.off_h3blk);
 
   const uint32_t lo = blockIdx.x * p.seg;
   const uint32_t hi = min(lo + p.seg, p.N);
-  uint32_t* seg = p.cand + static_cast<size_t>(blockIdx.x) * p.seg;
-  const uint32_t* su = reinterpret_cast<const uint32_t*>(p.s);
+  uint32_t wl, wh;
+  warp_slice(lo, hi, &wl, &wh);
+  uint2* wseg = p.cand + wl;   // this warp's candidate pairs
+  const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const bool none = p.k == 0;
   if (p.test_stall && blockIdx.x == 0) return;
   for (int i = threadIdx.x; i < kHeadWin; i += kThr) win[i] = 0;
@@ -469,20 +490,17 @@ __global__ void __launch_bounds__(kThr, 2)
   __syncthreads();
   const uint32_t ub1 = static_cast<uint32_t>(b1);
   HeadCounter hc(lo / p.n_c, p.n_c, p.n_heads, win, heads);
-  const uint32_t n_cand =
-      mask_pass(p.s, lo, hi, ub1, none, p.vec != 0, p.vec_keep != 0, p.keep, seg, hi - lo,
-                h2, tmp, [&](uint32_t f) { hc.add(f); });
+  const uint32_t n_w = mask_pass(p.s, wl, wh, Round1(b1, none), p.vec != 0, p.vec_keep != 0,
+                                 p.keep, wseg, h2, hc);
   hc.flush();
   __syncthreads();
   for (int i = threadIdx.x; i < kBins2; i += kThr)
     if (h2[i]) atomicAdd(g2 + i, h2[i]);
-  if (threadIdx.x == 0) blk_cand[blockIdx.x] = n_cand;
   if (!grid_barrier(sy, status, p.timeout_ns)) return;
 
   uint32_t tau = 0x7F800000u;
   uint64_t take_eq = 0;
   bool rank_ties = false;
-  uint64_t tie_base = 0;
   if (!none) {
     // ---------------------------------------------------------- D: round 2, round-3 histogram
     int b2;
@@ -493,13 +511,15 @@ __global__ void __launch_bounds__(kThr, 2)
     uint32_t* h3 = h1;   // reuse
     for (int i = threadIdx.x; i < kBins3; i += kThr) h3[i] = 0;
     __syncthreads();
-    for (uint32_t j = threadIdx.x; j < n_cand; j += kThr) {
-      const uint32_t w = __ldg(su + seg[j]);
+    for (uint32_t j = lane; j < n_w; j += 32) {
+      const uint32_t w = wseg[j].y;
       if ((w >> kShift2) == (pre2 >> kShift2)) atomicAdd(&h3[w & (kBins3 - 1)], 1u);
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < kBins3; i += kThr)
+    for (int i = threadIdx.x; i < kBins3; i += kThr) {   // kept for the tie ranks of E
+      h3blk[static_cast<size_t>(blockIdx.x) * kBins3 + i] = h3[i];
       if (h3[i]) atomicAdd(g3 + i, h3[i]);
+    }
     if (!grid_barrier(sy, status, p.timeout_ns)) return;
 
     // ---------------------------------------------------------- E: threshold, tie ranks
@@ -513,40 +533,43 @@ __global__ void __launch_bounds__(kThr, 2)
     HeadCounter hf(lo / p.n_c, p.n_c, p.n_heads, win, heads);
     if (!rank_ties) {
       // ---------------------------------------------------------- F: kept candidates
-      for (uint32_t j = threadIdx.x; j < n_cand; j += kThr) {
-        const uint32_t f = seg[j];
-        if (__ldg(su + f) >= tau && in_bounds(f >= lo && f < hi)) {
-          p.keep[f] = 1;
-          hf.add(f);
+      for (uint32_t j = lane; j < n_w; j += 32) {
+        const uint2 c = wseg[j];
+        if (c.y >= tau && in_bounds(c.x >= lo && c.x < hi)) {
+          p.keep[c.x] = 1;
+          hf.add(c.x);
         }
       }
     } else {
-      // Ties straddle the threshold: rank them in flat order.  Each thread takes a
-      // contiguous run of the block's candidates (which are in flat order), so one
-      // block scan of per-thread tie counts and one scan over the blocks give
-      // every tie its global rank.
-      const uint32_t run = (n_cand + kThr - 1) / kThr;
-      const uint32_t j0 = min(threadIdx.x * run, n_cand), j1 = min(j0 + run, n_cand);
-      uint32_t c = 0;
-      for (uint32_t j = j0; j < j1; ++j) c += (__ldg(su + seg[j]) == tau);
-      uint32_t tot;
-      const uint32_t mine_before = block_excl(c, tmp, &tot);
-      if (threadIdx.x == 0) blk_tie[blockIdx.x] = tot;
-      if (!grid_barrier(sy, status, p.timeout_ns)) return;
+      // Ties straddle the threshold: rank them in flat order.  Ties in earlier
+      // blocks come from their stored round-3 histograms (bin b3 holds exactly
+      // the scores equal to tau), ties in earlier warps from per-warp counts,
+      // and a ballot walk over the warp's pairs ranks the rest.
       uint32_t part = 0;
-      for (uint32_t b = threadIdx.x; b < blockIdx.x; b += kThr) part += __ldcg(blk_tie + b);
+      for (uint32_t b = threadIdx.x; b < blockIdx.x; b += kThr)
+        part += __ldcg(h3blk + static_cast<size_t>(b) * kBins3 + b3);
+      uint32_t tot;
       block_excl(part, tmp, &tot);
-      tie_base = tot;
+      uint32_t c = 0;
+      for (uint32_t j = lane; j < n_w; j += 32) c += (wseg[j].y == tau);
+      c = __reduce_add_sync(0xffffffffu, c);
+      if (lane == 0) wtie[warp] = c;
+      __syncthreads();
+      uint64_t rank = tot;
+      for (uint32_t v = 0; v < warp; ++v) rank += wtie[v];
       // ---------------------------------------------------------- F: kept candidates
-      uint64_t rank = tie_base + mine_before;
-      for (uint32_t j = j0; j < j1; ++j) {
-        const uint32_t f = seg[j];
-        const uint32_t w = __ldg(su + f);
-        bool kp = w > tau;
-        if (w == tau) kp = rank++ < take_eq;
-        if (kp && in_bounds(f >= lo && f < hi)) {
-          p.keep[f] = 1;
-          hf.add(f);
+      const uint32_t lt = (1u << lane) - 1u;
+      for (uint32_t j0 = 0; j0 < n_w; j0 += 32) {
+        const uint32_t j = j0 + lane;
+        const bool valid = j < n_w;
+        const uint2 e = valid ? wseg[j] : make_uint2(0u, 0u);
+        const bool tie = valid && e.y == tau;
+        const uint32_t m = __ballot_sync(0xffffffffu, tie);
+        const bool kp = valid && (e.y > tau || (tie && rank + __popc(m & lt) < take_eq));
+        rank += __popc(m);
+        if (kp && in_bounds(e.x >= lo && e.x < hi)) {
+          p.keep[e.x] = 1;
+          hf.add(e.x);
         }
       }
     }
@@ -586,17 +609,19 @@ __global__ void __launch_bounds__(kThr, 2)
 // on the candidates, then the kept candidates.  offsets[h] = h * k.
 __global__ void __launch_bounds__(kThr, 2)
     select_per_head_kernel(const float* __restrict__ s, uint32_t n_c, uint32_t n_heads,
-                           uint32_t k, uint8_t* keep, int64_t* offsets, uint32_t* cand,
-                           int vec, int vec_keep) {
+                           uint32_t k, uint8_t* keep, int64_t* offsets, uint2* cand, int vec,
+                           int vec_keep) {
   __shared__ uint32_t h1[kBins1];
   __shared__ uint32_t h2[kBins2];
-  __shared__ uint32_t tmp[2 * (kThr / 32)];
+  __shared__ uint32_t wtie[kWarps];
   const uint32_t head = blockIdx.x;
   const size_t lo = static_cast<size_t>(head) * n_c;
   const float* sh = s + lo;
   uint8_t* kh = keep + lo;
-  uint32_t* seg = cand + lo;
-  const uint32_t* su = reinterpret_cast<const uint32_t*>(sh);
+  const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t wl, wh;
+  warp_slice(0, n_c, &wl, &wh);
+  uint2* wseg = cand + lo + wl;   // this warp's candidate pairs (indices within the head)
   const bool none = k == 0;
   // rows of this head start on 16 bytes only when n_c is a multiple of 4
   const bool v4 = vec && (n_c % 4 == 0);
@@ -620,8 +645,8 @@ __global__ void __launch_bounds__(kThr, 2)
   const uint32_t ub1 = static_cast<uint32_t>(b1);
   for (int i = threadIdx.x; i < kBins2; i += kThr) h2[i] = 0;
   __syncthreads();
-  const uint32_t n_cand = mask_pass(sh, 0, n_c, ub1, none, v4, k4, kh, seg, n_c, h2, tmp,
-                                    [](uint32_t) {});
+  NoCounter nc;
+  const uint32_t n_w = mask_pass(sh, wl, wh, Round1(b1, none), v4, k4, kh, wseg, h2, nc);
   __syncthreads();
   if (none) return;
   int b2;
@@ -632,8 +657,8 @@ __global__ void __launch_bounds__(kThr, 2)
   uint32_t* h3 = h1;
   for (int i = threadIdx.x; i < kBins3; i += kThr) h3[i] = 0;
   __syncthreads();
-  for (uint32_t j = threadIdx.x; j < n_cand; j += kThr) {
-    const uint32_t w = __ldg(su + seg[j]);
+  for (uint32_t j = lane; j < n_w; j += 32) {
+    const uint32_t w = wseg[j].y;
     if ((w >> kShift2) == (pre2 >> kShift2)) atomicAdd(&h3[w & (kBins3 - 1)], 1u);
   }
   __syncthreads();
@@ -644,26 +669,31 @@ __global__ void __launch_bounds__(kThr, 2)
   const uint64_t take_eq = k_rem;
   const bool rank_ties = take_eq < h3[b3];
   if (!rank_ties) {
-    for (uint32_t j = threadIdx.x; j < n_cand; j += kThr) {
-      const uint32_t f = seg[j];
-      if (__ldg(su + f) >= tau && in_bounds(f < n_c)) kh[f] = 1;
+    for (uint32_t j = lane; j < n_w; j += 32) {
+      const uint2 c = wseg[j];
+      if (c.y >= tau && in_bounds(c.x < n_c)) kh[c.x] = 1;
     }
     return;
   }
-  // ties straddle the threshold: contiguous runs of candidates per thread, one
-  // block scan of the per-thread tie counts gives each tie its rank in position order
-  const uint32_t run = (n_cand + kThr - 1) / kThr;
-  const uint32_t j0 = min(threadIdx.x * run, n_cand), j1 = min(j0 + run, n_cand);
+  // ties straddle the threshold: per-warp tie counts give each warp the rank
+  // of its first tie in position order, and a ballot walk ranks the rest
   uint32_t c = 0;
-  for (uint32_t j = j0; j < j1; ++j) c += (__ldg(su + seg[j]) == tau);
-  uint32_t tot;
-  uint64_t rank = block_excl(c, tmp, &tot);
-  for (uint32_t j = j0; j < j1; ++j) {
-    const uint32_t f = seg[j];
-    const uint32_t w = __ldg(su + f);
-    bool kp = w > tau;
-    if (w == tau) kp = rank++ < take_eq;
-    if (kp && in_bounds(f < n_c)) kh[f] = 1;
+  for (uint32_t j = lane; j < n_w; j += 32) c += (wseg[j].y == tau);
+  c = __reduce_add_sync(0xffffffffu, c);
+  if (lane == 0) wtie[warp] = c;
+  __syncthreads();
+  uint64_t rank = 0;
+  for (uint32_t v = 0; v < warp; ++v) rank += wtie[v];
+  const uint32_t lt = (1u << lane) - 1u;
+  for (uint32_t j0 = 0; j0 < n_w; j0 += 32) {
+    const uint32_t j = j0 + lane;
+    const bool valid = j < n_w;
+    const uint2 e = valid ? wseg[j] : make_uint2(0u, 0u);
+    const bool tie = valid && e.y == tau;
+    const uint32_t m = __ballot_sync(0xffffffffu, tie);
+    const bool kp = valid && (e.y > tau || (tie && rank + __popc(m & lt) < take_eq));
+    rank += __popc(m);
+    if (kp && in_bounds(e.x < n_c)) kh[e.x] = 1;
   }
 }
 
@@ -693,13 +723,13 @@ cudaError_t coop_capacity(int* out) {
 size_t select_fused_ws_bytes(int64_t N, int64_t n_heads) { return layout(N, n_heads).total; }
 
 size_t select_per_head_ws_bytes(int64_t n_heads, int64_t n_c) {
-  return up256(static_cast<size_t>(n_heads) * static_cast<size_t>(n_c) * 4);
+  return up256(static_cast<size_t>(n_heads) * static_cast<size_t>(n_c) * 8);
 }
 
 cudaError_t launch_select_per_head(const SelectArgs& a, cudaStream_t s, int* launches) {
   select_per_head_kernel<<<static_cast<unsigned>(a.n_heads), kThr, 0, s>>>(
       a.scores, static_cast<uint32_t>(a.n_c), static_cast<uint32_t>(a.n_heads),
-      static_cast<uint32_t>(a.k), a.keep, a.offsets, static_cast<uint32_t*>(a.ws),
+      static_cast<uint32_t>(a.k), a.keep, a.offsets, static_cast<uint2*>(a.ws),
       reinterpret_cast<uintptr_t>(a.scores) % 16 == 0 ? 1 : 0,
       reinterpret_cast<uintptr_t>(a.keep) % 4 == 0 ? 1 : 0);
   if (launches) *launches += 1;
@@ -715,10 +745,9 @@ cudaError_t launch_select_fused(const SelectArgs& a, uint64_t timeout_ns, int te
   if (e != cudaSuccess) return e;
   const int64_t N = a.N;
   // Blocks: enough to fill the GPU, but no block with less than one tile.
-  const int64_t want = (N + kTile - 1) / kTile;
-  const int P = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(cap, want)));
+  const int P = static_cast<int>(std::min<int64_t>(cap, max_blocks(N)));
   int64_t seg = (N + P - 1) / P;
-  seg = (seg + 3) / 4 * 4;
+  seg = (seg + 127) / 128 * 128;   // ranges start on 512 bytes
   const int P_used = static_cast<int>((N + seg - 1) / seg);
   const Layout L = layout(N, a.n_heads);
   uint8_t* ws = static_cast<uint8_t*>(a.ws);
@@ -734,7 +763,7 @@ cudaError_t launch_select_fused(const SelectArgs& a, uint64_t timeout_ns, int te
   p.offsets = a.offsets;
   p.threshold = a.threshold;
   p.ws = ws;
-  p.cand = reinterpret_cast<uint32_t*>(ws + L.off_cand);
+  p.cand = reinterpret_cast<uint2*>(ws + L.off_cand);
   p.seg = static_cast<uint32_t>(seg);
   p.timeout_ns = timeout_ns;
   p.vec = reinterpret_cast<uintptr_t>(a.scores) % 16 == 0 ? 1 : 0;   // ranges start on 4 scores

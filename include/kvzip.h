@@ -172,8 +172,9 @@ void kvzip_set_test_stall(int on);
  * [0, 1] or N < 0.  r is the KEPT fraction ("30% cache ratio"). */
 int64_t kvzip_keep_count(double r, int64_t N);
 
-/* Bytes of workspace kvzip_select needs: about 4 * N bytes (a candidate
- * buffer of flat indices) plus ~40 KB and 4 bytes per head. */
+/* Bytes of workspace kvzip_select needs: about 8 * N bytes (a candidate
+ * buffer of (flat index, score bits) pairs) plus ~40 KB, 2 KB per 2048 scores
+ * up to 2 MB (per-block histograms) and 4 bytes per head. */
 size_t kvzip_select_workspace_size(int64_t N, int64_t n_heads);
 
 /*
@@ -362,7 +363,8 @@ kvzip_status kvzip_expand_keep(const uint8_t* keep_pos, const int64_t* pos_offse
                                int64_t n_heads, int64_t n_c, uint8_t* keep, int64_t* offsets,
                                void* stream);
 
-/* Bytes of workspace kvzip_select_per_head needs. */
+/* Bytes of workspace kvzip_select_per_head needs: 8 * n_heads * n_c (a
+ * candidate buffer of (position, score bits) pairs). */
 size_t kvzip_select_per_head_workspace_size(int64_t n_heads, int64_t n_c);
 
 /*
