@@ -3,9 +3,10 @@
 // The authors compute a context-independent head score as max_i S[:, :, i]
 // over the sequence dimension of the L x H x n_c score tensor (OpenReview
 // rebuttal, answer on how head-level scores were measured for the
-// DuoAttention comparison).  Scores are >= 0, so their IEEE bits order like
-// the values and the per-segment maxima combine with an integer atomicMax
-// into an output zeroed first (0.0f is a lower bound of every score).
+// DuoAttention comparison).  Scores are >= 0, so the bits of |s| (mag: -0.0
+// reads as 0.0) order like the values and the per-segment maxima combine with
+// an integer atomicMax into an output zeroed first (0.0f is a lower bound of
+// every score).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -28,7 +29,7 @@ __global__ void __launch_bounds__(kHeadThreads)
   const float* base = s + h * n_c;
   uint32_t m = 0;
   for (int64_t j = j0 + threadIdx.x; j < j1; j += kHeadThreads) {
-    const uint32_t u = __float_as_uint(__ldcs(base + j));
+    const uint32_t u = mag(__float_as_uint(__ldcs(base + j)));
     m = u > m ? u : m;
   }
   m = __reduce_max_sync(0xffffffffu, m);
@@ -81,7 +82,8 @@ __global__ void __launch_bounds__(kHeadThreads)
     for (int q = 0; q < 4; ++q)   // zeros never raise a maximum of scores >= 0
       u[q] = (i + q * kHeadThreads < n4) ? __ldcs(b4 + i + q * kHeadThreads) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) m = max(m, max(max(u[q].x, u[q].y), max(u[q].z, u[q].w)));
+    for (int q = 0; q < 4; ++q)
+      m = max(m, max(max(mag(u[q].x), mag(u[q].y)), max(mag(u[q].z), mag(u[q].w))));
   }
   m = __reduce_max_sync(0xffffffffu, m);
   __shared__ uint32_t red[kHeadThreads / 32];
@@ -110,10 +112,10 @@ __global__ void __launch_bounds__(256)
 #pragma unroll 4
   for (int64_t h = h0; h < h1; ++h, p += row4) {
     const uint4 u = __ldcs(p);
-    m.x = max(m.x, u.x);
-    m.y = max(m.y, u.y);
-    m.z = max(m.z, u.z);
-    m.w = max(m.w, u.w);
+    m.x = max(m.x, mag(u.x));
+    m.y = max(m.y, mag(u.y));
+    m.z = max(m.z, mag(u.z));
+    m.w = max(m.w, mag(u.w));
   }
   uint32_t* t = tok + 4 * j4;
   atomicMax(t + 0, m.x);

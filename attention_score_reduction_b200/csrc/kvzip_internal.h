@@ -157,4 +157,9 @@ cudaError_t bounds_flag_select_fused(unsigned int* out);
 cudaError_t bounds_flag_compact(unsigned int* out);
 cudaError_t bounds_flag_decode(unsigned int* out);
 
+// Scores are ranked by the bits of |s|: for s >= 0 the bit order is the value
+// order, and -0.0 ranks as 0.0 (its raw bits would rank above every score).
+// Every kernel that compares or orders score bits reads them through mag.
+__host__ __device__ __forceinline__ uint32_t mag(uint32_t w) { return w & 0x7FFFFFFFu; }
+
 }  // namespace kvzip

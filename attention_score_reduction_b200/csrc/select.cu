@@ -6,8 +6,9 @@
 // budgets; rebuttal: S has shape L x H x n_c).  The kept set is the k largest
 // scores; equal scores are taken lowest flat index first, so the mask is unique.
 //
-// Scores are finite and >= 0, so their IEEE bit patterns, read as uint32, sort
-// like the values.  The threshold tau (the k-th largest bit pattern) is found
+// Scores are finite and >= 0, so the bit patterns of |s| (mag: -0.0 reads as
+// 0.0), read as uint32, sort like the values.  The threshold tau (the k-th
+// largest such pattern) is found
 // by a three-round radix select on 13 + 10 + 9 bits; every round is one
 // histogram pass over HBM plus a one-block pick, all on the stream with no
 // host round trip.  A mask pass then writes keep[f] and per-block kept counts;
@@ -102,16 +103,18 @@ __device__ __forceinline__ void hist_count(const float* __restrict__ s, int64_t 
   // two independent 16-byte loads in flight per thread
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
        i += 2 * stride) {
+    const bool in1 = i + stride < n4;
     const uint4 u0 = __ldcs(s4 + i);
-    const uint4 u1 = (i + stride < n4) ? __ldcs(s4 + i + stride) : make_uint4(~0u, ~0u, ~0u, ~0u);
-    const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+    const uint4 u1 = in1 ? __ldcs(s4 + i + stride) : make_uint4(0, 0, 0, 0);
+    const uint32_t w[8] = {mag(u0.x), mag(u0.y), mag(u0.z), mag(u0.w),
+                           mag(u1.x), mag(u1.y), mag(u1.z), mag(u1.w)};
 #pragma unroll
-    for (int e = 0; e < 8; ++e)   // all-ones (a NaN pattern) never matches a prefix of a score
-      if (w[e] != ~0u && (w[e] & PM) == prefix) atomicAdd(&h[(w[e] >> SH) & (NB - 1)], 1u);
+    for (int e = 0; e < 8; ++e)
+      if ((e < 4 || in1) && (w[e] & PM) == prefix) atomicAdd(&h[(w[e] >> SH) & (NB - 1)], 1u);
   }
   for (int64_t i = 4 * n4 + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < N;
        i += stride) {
-    const uint32_t w = __float_as_uint(s[i]);
+    const uint32_t w = mag(__float_as_uint(s[i]));
     if ((w & PM) == prefix) atomicAdd(&h[(w >> SH) & (NB - 1)], 1u);
   }
 }
@@ -236,7 +239,7 @@ __global__ void __launch_bounds__(kSelThreads)
   const uint32_t tau = st->tau;
   uint32_t c = 0;
   for (int64_t j = j0 + threadIdx.x; j < j1; j += kSelThreads)
-    c += (__float_as_uint(base[j]) == tau);
+    c += (mag(__float_as_uint(base[j])) == tau);
   __shared__ uint32_t red[kSelThreads / 32];
   c = __reduce_add_sync(0xffffffffu, c);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = c;
@@ -263,10 +266,12 @@ __global__ void __launch_bounds__(kSelThreads)
   const uint32_t tau = st->tau;
   uint32_t c = 0;
   for (int64_t i = threadIdx.x; i < n4; i += 2 * kSelThreads) {
+    const bool in1 = i + kSelThreads < n4;
     const uint4 u0 = __ldcs(b4 + i);
-    const uint4 u1 = (i + kSelThreads < n4) ? __ldcs(b4 + i + kSelThreads) : make_uint4(~0u, ~0u, ~0u, ~0u);
-    c += (u0.x == tau) + (u0.y == tau) + (u0.z == tau) + (u0.w == tau) + (u1.x == tau) +
-         (u1.y == tau) + (u1.z == tau) + (u1.w == tau);
+    const uint4 u1 = in1 ? __ldcs(b4 + i + kSelThreads) : make_uint4(0, 0, 0, 0);
+    c += (mag(u0.x) == tau) + (mag(u0.y) == tau) + (mag(u0.z) == tau) + (mag(u0.w) == tau);
+    if (in1)
+      c += (mag(u1.x) == tau) + (mag(u1.y) == tau) + (mag(u1.z) == tau) + (mag(u1.w) == tau);
   }
   __shared__ uint32_t red[kSelThreads / 32];
   c = __reduce_add_sync(0xffffffffu, c);
@@ -280,7 +285,7 @@ __global__ void __launch_bounds__(kSelThreads)
 }
 
 __device__ __forceinline__ uint32_t mask4(uint4 u, uint32_t tau, bool eq_keeps) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  const uint32_t w[4] = {mag(u.x), mag(u.y), mag(u.z), mag(u.w)};
   uint32_t m = 0;
 #pragma unroll
   for (int e = 0; e < 4; ++e)
@@ -325,7 +330,7 @@ __global__ void __launch_bounds__(kSelThreads)
       const int64_t i = ib + threadIdx.x;
       const bool in = i < n4;
       const uint4 u = in ? __ldcs(b4 + i) : make_uint4(0, 0, 0, 0);
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      const uint32_t w[4] = {mag(u.x), mag(u.y), mag(u.z), mag(u.w)};
       uint32_t c_eq = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) c_eq += (in && w[e] == tau);
@@ -412,7 +417,7 @@ __global__ void __launch_bounds__(kSelThreads)
   for (int64_t jb = j0; jb < j1; jb += kSelThreads) {
     const int64_t j = jb + threadIdx.x;
     const bool in = j < j1;
-    const uint32_t u = in ? __float_as_uint(base[j]) : 0u;
+    const uint32_t u = in ? mag(__float_as_uint(base[j])) : 0u;
     bool k = in && !none && u > tau;
     const bool eq = in && !none && u == tau;
     if (!rank_ties) {
@@ -593,7 +598,7 @@ __global__ void __launch_bounds__(kSelThreads)
   uint32_t c = 0;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < N;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    c += (__float_as_uint(s[i]) == tau);
+    c += (mag(__float_as_uint(s[i])) == tau);
   c = __reduce_add_sync(0xffffffffu, c);
   if ((threadIdx.x & 31) == 0 && c) atomicAdd(n_ties, static_cast<unsigned long long>(c));
 }

@@ -196,6 +196,58 @@ __device__ __forceinline__ uint32_t block_excl(uint32_t v, uint32_t* tmp, uint32
   return before + inc - v;
 }
 
+// |x| - t on the FMA pipe, IEEE subnormals kept: negative iff |x| < t (for t
+// finite or +inf and x not NaN; a NaN gives a positive NaN).
+__device__ __forceinline__ float abs_minus(uint32_t x, float t) {
+  float r;
+  asm("{\n\t.reg .f32 a;\n\tabs.f32 a, %1;\n\tsub.rn.f32 %0, a, %2;\n\t}"
+      : "=f"(r)
+      : "f"(__uint_as_float(x)), "f"(t));
+  return r;
+}
+
+// Byte e = 0xFF if the e-th argument's sign bit is set, else 0x00 (byte
+// permutes with sign replication, then one merge).
+__device__ __forceinline__ uint32_t sign_bytes4(float a, float b, float c, float d) {
+  uint32_t lo, hi, r;
+  asm("prmt.b32 %0, %1, %2, 0x00FB;" : "=r"(lo) : "r"(__float_as_uint(a)), "r"(__float_as_uint(b)));
+  asm("prmt.b32 %0, %1, %2, 0xFB00;" : "=r"(hi) : "r"(__float_as_uint(c)), "r"(__float_as_uint(d)));
+  asm("prmt.b32 %0, %1, %2, 0x7610;" : "=r"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+
+// Four 16-byte loads issued back to back from one statement, so all four are
+// in flight before the first is used: scores p[0..3], p[128..131],
+// p[256..259], p[384..387] (512-byte steps; ld.global.cs, evict first) or,
+// for ld4_nc_tile, four block tiles apart (read-only path).
+__device__ __forceinline__ void ld4_cs(const uint4* p, uint4 (&a)[4]) {
+  asm volatile(
+      "{\n\t"
+      "ld.global.cs.v4.u32 {%0,%1,%2,%3}, [%16];\n\t"
+      "ld.global.cs.v4.u32 {%4,%5,%6,%7}, [%16+512];\n\t"
+      "ld.global.cs.v4.u32 {%8,%9,%10,%11}, [%16+1024];\n\t"
+      "ld.global.cs.v4.u32 {%12,%13,%14,%15}, [%16+1536];\n\t}"
+      : "=r"(a[0].x), "=r"(a[0].y), "=r"(a[0].z), "=r"(a[0].w), "=r"(a[1].x), "=r"(a[1].y),
+        "=r"(a[1].z), "=r"(a[1].w), "=r"(a[2].x), "=r"(a[2].y), "=r"(a[2].z), "=r"(a[2].w),
+        "=r"(a[3].x), "=r"(a[3].y), "=r"(a[3].z), "=r"(a[3].w)
+      : "l"(p)
+      : "memory");
+}
+static_assert(kTile * 4 == 8192, "ld4_nc_tile's offsets are four block tiles");
+__device__ __forceinline__ void ld4_nc_tile(const uint4* p, uint4 (&a)[4]) {
+  asm volatile(
+      "{\n\t"
+      "ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%16];\n\t"
+      "ld.global.nc.v4.u32 {%4,%5,%6,%7}, [%16+8192];\n\t"
+      "ld.global.nc.v4.u32 {%8,%9,%10,%11}, [%16+16384];\n\t"
+      "ld.global.nc.v4.u32 {%12,%13,%14,%15}, [%16+24576];\n\t}"
+      : "=r"(a[0].x), "=r"(a[0].y), "=r"(a[0].z), "=r"(a[0].w), "=r"(a[1].x), "=r"(a[1].y),
+        "=r"(a[1].z), "=r"(a[1].w), "=r"(a[2].x), "=r"(a[2].y), "=r"(a[2].z), "=r"(a[2].w),
+        "=r"(a[3].x), "=r"(a[3].y), "=r"(a[3].z), "=r"(a[3].w)
+      : "l"(p)
+      : "memory");
+}
+
 // Round-1 histogram of the top 13 bits of the scores [lo, hi) of s (indices
 // relative to s) into shared memory: four 16-byte loads in flight per thread.
 __device__ __forceinline__ void hist_top(const float* __restrict__ s, uint32_t lo, uint32_t hi,
@@ -206,14 +258,13 @@ __device__ __forceinline__ void hist_top(const float* __restrict__ s, uint32_t l
     const uint32_t i0 = g0 + 4 * threadIdx.x;
     if (vec && i0 + 3 * kTile + 3 < hi) {
       uint4 a[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) a[q] = __ldg(s4 + (i0 + q * kTile) / 4);
+      ld4_nc_tile(s4 + i0 / 4, a);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        atomicAdd(&h1[a[q].x >> kShift1], 1u);
-        atomicAdd(&h1[a[q].y >> kShift1], 1u);
-        atomicAdd(&h1[a[q].z >> kShift1], 1u);
-        atomicAdd(&h1[a[q].w >> kShift1], 1u);
+        atomicAdd(&h1[mag(a[q].x) >> kShift1], 1u);
+        atomicAdd(&h1[mag(a[q].y) >> kShift1], 1u);
+        atomicAdd(&h1[mag(a[q].z) >> kShift1], 1u);
+        atomicAdd(&h1[mag(a[q].w) >> kShift1], 1u);
       }
     } else {
 #pragma unroll
@@ -221,7 +272,7 @@ __device__ __forceinline__ void hist_top(const float* __restrict__ s, uint32_t l
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const uint32_t f = i0 + q * kTile + e;
-          if (f < hi) atomicAdd(&h1[__ldg(su + f) >> kShift1], 1u);
+          if (f < hi) atomicAdd(&h1[mag(__ldg(su + f)) >> kShift1], 1u);
         }
     }
   }
@@ -235,26 +286,38 @@ __device__ __forceinline__ void warp_slice(uint32_t lo, uint32_t hi, uint32_t* w
   *wh = min(*wl + len, hi);
 }
 
-// Round-1 decision per score, from its bits w (scores >= 0 order like their
-// bits): kept iff w > lim (its 13-bit bin is above b1); a candidate iff
-// w - base < width (its bin is b1).  With k = 0 nothing is kept or a candidate.
+// Round-1 decision per score, from w = mag(bits): kept iff w > lim (its
+// 13-bit bin is above b1); a candidate iff w - base < width (its bin is b1).
+// With k = 0 nothing is kept or a candidate.  When the first value of bin
+// b1 + 1 is finite or +inf (fast), the same decisions come from float
+// subtractions on the FMA pipe: kept iff |s| >= t_keep, below bin b1 iff
+// |s| < t_base.  For |s| not NaN this is the bit order; a NaN's bits lie above
+// +inf and its difference is a positive NaN, so it counts as kept either way.
 struct Round1 {
   uint32_t lim, base, width;
+  bool fast;
+  float t_keep, t_base;
   __device__ Round1(int b1, bool none) {
     const uint32_t b = static_cast<uint32_t>(b1);
     lim = none ? 0xFFFFFFFFu : ((b << kShift1) | ((1u << kShift1) - 1));
     base = none ? 0u : (b << kShift1);
     width = none ? 0u : (1u << kShift1);
+    fast = !none && b + 1 <= (0x7F800000u >> kShift1);
+    t_keep = __uint_as_float(fast ? (b + 1) << kShift1 : 0u);
+    t_base = __uint_as_float(fast ? b << kShift1 : 0u);
   }
 };
 
 // Second pass over a warp's slice [wl, wh) of s, 512 scores per step (four
 // 16-byte loads in flight per lane): the final mask byte of every score
 // outside bin b1 (0 for candidates, set later), the candidates appended as
-// (flat index, bits) pairs to seg in flat order (positions from one warp scan
-// of per-load counts packed in bytes), their round-2 digits histogrammed into
-// h2, and cnt.add4(i, km) for each group of four scores at i with kept bits
-// km (in increasing i per lane).  Returns the warp's candidate count.
+// (flat index, mag bits) pairs to seg in flat order (positions from one warp
+// scan of per-load counts packed in bytes; each lane then walks its own
+// candidate bits), their round-2 digits histogrammed into h2, and each step's
+// kept scores passed to cnt.add_step.  Each group of four scores gets its
+// decisions as byte masks: on the fast path four float subtractions and the
+// sign bytes of their results, otherwise integer compares.  Returns the
+// warp's candidate count.
 template <class Counter>
 __device__ uint32_t mask_pass(const float* __restrict__ s, uint32_t wl, uint32_t wh,
                               const Round1 r1, bool vec, bool vec_keep, uint8_t* keep,
@@ -265,53 +328,78 @@ __device__ uint32_t mask_pass(const float* __restrict__ s, uint32_t wl, uint32_t
   uint32_t n_w = 0;   // warp-uniform
   for (uint32_t g0 = wl; g0 < wh; g0 += kWarpStep) {
     const uint32_t ib = g0 + 4 * lane;   // this lane's first score of load 0
+    const bool full = g0 + kWarpStep <= wh;   // warp-uniform
     uint4 a[4];
+    if (vec && full) {
+      ld4_cs(s4 + ib / 4, a);
+    } else {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {        // four loads in flight
-      const uint32_t i0 = ib + q * 128;
-      if (vec && i0 + 3 < wh) {
-        a[q] = __ldcs(s4 + i0 / 4);
-      } else {
-        a[q].x = (i0 + 0 < wh) ? __ldcs(su + i0 + 0) : 0u;
-        a[q].y = (i0 + 1 < wh) ? __ldcs(su + i0 + 1) : 0u;
-        a[q].z = (i0 + 2 < wh) ? __ldcs(su + i0 + 2) : 0u;
-        a[q].w = (i0 + 3 < wh) ? __ldcs(su + i0 + 3) : 0u;
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t i0 = ib + q * 128;
+        if (vec && i0 + 3 < wh) {
+          a[q] = __ldcs(s4 + i0 / 4);
+        } else {
+          a[q].x = (i0 + 0 < wh) ? __ldcs(su + i0 + 0) : 0u;
+          a[q].y = (i0 + 1 < wh) ? __ldcs(su + i0 + 1) : 0u;
+          a[q].z = (i0 + 2 < wh) ? __ldcs(su + i0 + 2) : 0u;
+          a[q].w = (i0 + 3 < wh) ? __ldcs(su + i0 + 3) : 0u;
+        }
       }
     }
-    uint32_t cm = 0, packed = 0;   // candidate bits (4q + e); candidates per load, one byte each
+    uint32_t cw[4], kws[4];   // candidate and kept byte masks per load
+    uint32_t any = 0, kacc = 0;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const uint32_t i0 = ib + q * 128;
-      const uint32_t w[4] = {a[q].x, a[q].y, a[q].z, a[q].w};
-      const uint32_t n_in = i0 < wh ? min(wh - i0, 4u) : 0u;
-      const uint32_t vm = (1u << n_in) - 1u;
-      uint32_t km = 0, cq = 0;
+      uint32_t kw, c;
+      if (r1.fast) {
+        const uint32_t nk = sign_bytes4(abs_minus(a[q].x, r1.t_keep), abs_minus(a[q].y, r1.t_keep),
+                                        abs_minus(a[q].z, r1.t_keep), abs_minus(a[q].w, r1.t_keep));
+        const uint32_t nb = sign_bytes4(abs_minus(a[q].x, r1.t_base), abs_minus(a[q].y, r1.t_base),
+                                        abs_minus(a[q].z, r1.t_base), abs_minus(a[q].w, r1.t_base));
+        kw = ~nk & 0x01010101u;        // not below bin b1 + 1
+        c = nk & ~nb & 0x01010101u;    // below bin b1 + 1, not below bin b1
+      } else {
+        const uint32_t w[4] = {mag(a[q].x), mag(a[q].y), mag(a[q].z), mag(a[q].w)};
+        uint32_t km = 0, cq = 0;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        km |= static_cast<uint32_t>(w[e] > r1.lim) << e;
-        cq |= static_cast<uint32_t>(w[e] - r1.base < r1.width) << e;
+        for (int e = 0; e < 4; ++e) {
+          km |= static_cast<uint32_t>(w[e] > r1.lim) << e;
+          cq |= static_cast<uint32_t>(w[e] - r1.base < r1.width) << e;
+        }
+        // bit e to byte e (the shifted copies do not overlap, so no carries)
+        kw = (km * 0x00204081u) & 0x01010101u;
+        c = (cq * 0x00204081u) & 0x01010101u;
       }
-      km &= vm;
-      cq &= vm;
+      const uint32_t n_in = full ? 4u : (i0 < wh ? min(wh - i0, 4u) : 0u);
+      if (!full) {
+        const uint32_t bm = n_in == 4 ? ~0u : (1u << (8 * n_in)) - 1u;
+        kw &= bm;
+        c &= bm;
+      }
       if (vec_keep && n_in == 4) {
-        // bit e of km to bit 8e (the shifted copies of km do not overlap, so no carries)
-        *reinterpret_cast<uint32_t*>(keep + i0) = (km * 0x00204081u) & 0x01010101u;
+        *reinterpret_cast<uint32_t*>(keep + i0) = kw;
       } else {
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          if (e < static_cast<int>(n_in)) keep[i0 + e] = static_cast<uint8_t>((km >> e) & 1u);
+          if (e < static_cast<int>(n_in)) keep[i0 + e] = static_cast<uint8_t>((kw >> (8 * e)) & 1u);
       }
-      if (cq) {
+      if (c) {
+        const uint32_t w[4] = {a[q].x, a[q].y, a[q].z, a[q].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          if ((cq >> e) & 1u) atomicAdd(&h2[(w[e] >> kShift2) & (kBins2 - 1)], 1u);
+          if ((c >> (8 * e)) & 1u) atomicAdd(&h2[(mag(w[e]) >> kShift2) & (kBins2 - 1)], 1u);
       }
-      cnt.add4(i0, km);
-      cm |= cq << (4 * q);
-      packed |= static_cast<uint32_t>(__popc(cq)) << (8 * q);
+      kws[q] = kw;
+      kacc += kw;               // bytes <= 4: no carries
+      cw[q] = c;
+      any |= c;
     }
-    if (__any_sync(0xffffffffu, cm != 0)) {
-      // per-load counts are <= 128 per warp, so the byte lanes of the scan never carry
+    cnt.add_step(g0, min(g0 + kWarpStep, wh), ib, kws, (kacc * 0x01010101u) >> 24);
+    if (__any_sync(0xffffffffu, any != 0)) {
+      // candidates per load, one byte each; <= 128 per warp, so the scan's bytes never carry
+      const uint32_t packed = __popc(cw[0]) | (__popc(cw[1]) << 8) | (__popc(cw[2]) << 16) |
+                              (__popc(cw[3]) << 24);
       uint32_t inc = packed;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -321,19 +409,27 @@ __device__ uint32_t mask_pass(const float* __restrict__ s, uint32_t wl, uint32_t
       const uint32_t tot = __shfl_sync(0xffffffffu, inc, 31), ex = inc - packed;
       const uint32_t t0 = tot & 0xFFu, t1 = (tot >> 8) & 0xFFu, t2 = (tot >> 16) & 0xFFu,
                      t3 = tot >> 24;
-      if (cm) {
-        const uint32_t before[4] = {0u, t0, t0 + t1, t0 + t1 + t2};
+      // this lane's candidates as bits 4q + e, written in that (flat) order
+      uint32_t m = 0;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t x = n_w + before[q] + ((ex >> (8 * q)) & 0xFFu);
-          const uint32_t w[4] = {a[q].x, a[q].y, a[q].z, a[q].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if ((cm >> (4 * q + e)) & 1u) {
-              if (in_bounds(x < wh - wl)) seg[x] = make_uint2(ib + q * 128 + e, w[e]);
-              ++x;
-            }
+      for (int q = 0; q < 4; ++q) m |= ((cw[q] * 0x01020408u) >> 24 & 0xFu) << (4 * q);
+      uint32_t prev_q = 0, x = n_w + (ex & 0xFFu);
+      while (m) {
+        const uint32_t b = __ffs(m) - 1;
+        m &= m - 1;
+        const uint32_t q = b >> 2;
+        if (q != prev_q) {   // first candidate of a later load: its base position
+          x = n_w + (q > 0 ? t0 : 0u) + (q > 1 ? t1 : 0u) + (q > 2 ? t2 : 0u) +
+              ((ex >> (8 * q)) & 0xFFu);
+          prev_q = q;
         }
+        const uint32_t e = b & 3u;
+        const uint32_t wq = q == 0 ? (e == 0 ? a[0].x : e == 1 ? a[0].y : e == 2 ? a[0].z : a[0].w)
+                          : q == 1 ? (e == 0 ? a[1].x : e == 1 ? a[1].y : e == 2 ? a[1].z : a[1].w)
+                          : q == 2 ? (e == 0 ? a[2].x : e == 1 ? a[2].y : e == 2 ? a[2].z : a[2].w)
+                                   : (e == 0 ? a[3].x : e == 1 ? a[3].y : e == 2 ? a[3].z : a[3].w);
+        if (in_bounds(x < wh - wl)) seg[x] = make_uint2(ib + q * 128 + e, mag(wq));
+        ++x;
       }
       n_w += t0 + t1 + t2 + t3;
     }
@@ -413,16 +509,19 @@ struct HeadCounter {
     }
     ++cnt;
   }
-  // The kept ones (bits of km) among the four scores i..i+3.
-  __device__ __forceinline__ void add4(uint32_t i, uint32_t km) {
-    if (!km) return;
-    if (i + 3 < end) {   // all four in the current head (indices only grow)
-      cnt += __popc(km);
+  // One mask-pass step of a lane: scores i + 128 q + e (q, e < 4) with kept
+  // bytes kw[q] (byte e = 1 if kept), n_kept of them; all in [lo, hi).
+  __device__ __forceinline__ void add_step(uint32_t lo, uint32_t hi, uint32_t i,
+                                           const uint32_t (&kw)[4], uint32_t n_kept) {
+    if (lo >= h * n_c && hi <= end) {   // the whole step lies in the current head
+      cnt += n_kept;
       return;
     }
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
-      if ((km >> e) & 1u) add(i + e);
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if ((kw[q] >> (8 * e)) & 1u) add(i + 128 * q + e);
   }
   __device__ __forceinline__ void flush() {
     if (!cnt) return;
@@ -435,7 +534,8 @@ struct HeadCounter {
 };
 
 struct NoCounter {
-  __device__ __forceinline__ void add4(uint32_t, uint32_t) {}
+  __device__ __forceinline__ void add_step(uint32_t, uint32_t, uint32_t, const uint32_t (&)[4],
+                                           uint32_t) {}
 };
 
 __global__ void __launch_bounds__(kThr, 2)

@@ -190,6 +190,53 @@ def test_select_no_scores(kz):
     del keep, s
 
 
+def _signed_zero_scores(n_heads, n_c, seed):
+    """Scores in {0.0, -0.0, 0.125, 0.5}: -0.0 equals 0.0, so at r = 0.5 the
+    threshold is 0 and the zeros of both signs tie, ranked by index."""
+    g = np.random.default_rng(seed)
+    s = g.choice(np.array([0.0, 0.125, 0.5], np.float32), size=(n_heads, n_c),
+                 p=[0.6, 0.25, 0.15])
+    s[(s == 0) & (g.random(s.shape) < 0.5)] = np.float32(-0.0)
+    assert np.signbit(s).any()
+    return s
+
+
+def _inf_scores(n_heads, n_c, seed):
+    """Uniform scores with 5% +inf: at r = 0.03 the threshold is +inf (the
+    k-th largest lies in the infinity bin), at r = 0.3 it is finite."""
+    g = np.random.default_rng(seed)
+    s = g.random((n_heads, n_c), dtype=np.float32)
+    s[g.random(s.shape) < 0.05] = np.inf
+    return s
+
+
+@pytest.mark.parametrize("make,rs", [(_signed_zero_scores, (0.3, 0.5, 0.9)),
+                                     (_inf_scores, (0.03, 0.3))], ids=["signed_zero", "inf"])
+def test_select_signed_zero_and_inf(kz, make, rs):
+    """Scores compare by value: -0.0 ranks as 0.0 (not by its raw bits, which
+    would rank it above every score), and +inf above every finite score, for
+    the global selection, the uniform per-head budgets and head/token scores."""
+    n_heads, n_c = 12, 5000
+    s = make(n_heads, n_c, seed=n_c)
+    sd = torch.from_numpy(s).cuda()
+    for r in rs:
+        k = kz.keep_count(r, s.size)
+        keep, off, thr = kz.select(sd.reshape(-1), k, n_heads)
+        keep_ref, off_ref, thr_ref = oracle.select(s.reshape(-1), k, n_heads)
+        assert np.array_equal(keep.cpu().numpy(), keep_ref), r
+        assert np.array_equal(off.cpu().numpy(), off_ref), r
+        assert float(thr.item()) == thr_ref
+        k_h = oracle.keep_count(r, n_c)
+        keep_h, off_h = kz.select_per_head(sd, k_h)
+        keep_h_ref, off_h_ref = oracle.select_per_head(s.reshape(-1), k_h, n_heads)
+        assert np.array_equal(keep_h.cpu().numpy(), keep_h_ref), r
+        assert np.array_equal(off_h.cpu().numpy(), off_h_ref), r
+    assert np.array_equal(kz.head_scores(sd).cpu().numpy(),
+                          oracle.head_scores(s, 1, n_heads).reshape(-1).astype(np.float32))
+    assert np.array_equal(kz.token_scores(sd).cpu().numpy(),
+                          oracle.token_scores(s).astype(np.float32))
+
+
 # ------------------------------------------------------------------ compaction
 
 @pytest.mark.parametrize("d", [128, 256])

@@ -97,6 +97,21 @@ def test_shard_protocol_matches_global_selection(kz, heads, n_c, levels):
             assert all(t == thr_ref for t in thr)
 
 
+def test_shard_protocol_signed_zero(kz):
+    """-0.0 ranks as 0.0 on every rank, as in the one-GPU selection."""
+    g = np.random.default_rng(3)
+    s = g.choice(np.array([0.0, 0.25], np.float32), size=(6, 700), p=[0.7, 0.3])
+    s[(s == 0) & (g.random(s.shape) < 0.5)] = np.float32(-0.0)
+    sd = torch.from_numpy(s).cuda()
+    parts = [sd[:2].contiguous(), sd[2:].contiguous()]
+    for r in (0.2, 0.5):
+        k = oracle.keep_count(r, s.size)
+        out, thr = _run_ranks(kz, parts, k)
+        keep_ref, off_ref, thr_ref = oracle.select(s.reshape(-1), k, 6)
+        assert np.array_equal(np.concatenate([o[0].cpu().numpy() for o in out]), keep_ref)
+        assert all(t == thr_ref for t in thr)
+
+
 def _gloo_worker(rank, world, port, q, heads, n_c, levels, r_keep):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     import datetime

@@ -64,6 +64,25 @@ def test_noalloc_select_matches_workspace_select_twice(lib):
             assert not bool(keep.any()) and float(thr.item()) == float("inf")
 
 
+def test_noalloc_select_signed_zero_and_inf(lib):
+    """The multi-launch selection ranks -0.0 as 0.0 and +inf above every finite
+    score, like the one-launch selection."""
+    L, kz = lib
+    import numpy as np
+    g = np.random.default_rng(9)
+    s = g.choice(np.array([0.0, 0.125, np.inf], np.float32), size=(8, 3000), p=[0.6, 0.3, 0.1])
+    s[(s == 0) & (g.random(s.shape) < 0.5)] = np.float32(-0.0)
+    sd = torch.from_numpy(s).reshape(-1).cuda()
+    for r in (0.05, 0.3, 0.7):
+        k = kz.keep_count(r, sd.numel())
+        keep_ref, off_ref, thr_ref = kz.select(sd, k, 8)
+        st, keep, off, thr = _noalloc(L, sd, k, 8)
+        torch.cuda.synchronize()
+        assert st == kz.OK
+        assert torch.equal(keep, keep_ref) and torch.equal(off, off_ref)
+        assert torch.equal(thr, thr_ref)
+
+
 def test_noalloc_select_rejects_oversize(lib):
     L, kz = lib
     s = torch.zeros(4, dtype=torch.float32, device="cuda")
