@@ -12,7 +12,7 @@
 //   C  every block reads its range again (read 2) and writes the final mask
 //      byte of every score outside bin b1 (kept iff its bin is above b1).  Each
 //      warp owns a contiguous slice of the block's range and appends the
-//      scores inside bin b1 (the candidates), as (flat index, score bits)
+//      scores inside bin b1 (the candidates), as (flat index, bits of |s|)
 //      pairs in flat order, to its own segment of a candidate buffer, placed
 //      by a warp scan (no block barrier in the streaming loop); their next 10
 //      bits are histogrammed; grid barrier.
@@ -26,6 +26,9 @@
 //   F  every block sets the mask of its kept candidates; grid barrier.
 //   G  block 0 turns the per-head kept counts into offsets and writes tau.
 //
+// Scores are ordered by the bits of |s| (mag): the value order for s >= 0,
+// with -0.0 equal to 0.0.
+//
 // Per-head kept counts are accumulated on the way (C and F) by run-length
 // counting per thread: a thread's scores are visited in increasing flat order,
 // so its head only changes at head boundaries.
@@ -35,7 +38,6 @@
 // records KVZIP_ERR_TIMEOUT in the workspace status word, raises an abort flag
 // that releases the other blocks, and the kernel returns with an incomplete
 // mask.
-#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -233,7 +235,7 @@ __device__ __forceinline__ void ld4_cs(const uint4* p, uint4 (&a)[4]) {
       : "l"(p)
       : "memory");
 }
-static_assert(kTile * 4 == 8192, "ld4_nc_tile's offsets are four block tiles");
+static_assert(kTile * 4 == 8192, "ld4_nc_tile's four loads are one block tile (8192 bytes) apart");
 __device__ __forceinline__ void ld4_nc_tile(const uint4* p, uint4 (&a)[4]) {
   asm volatile(
       "{\n\t"
