@@ -184,14 +184,17 @@ size_t kvzip_select_workspace_size(int64_t N, int64_t n_heads);
  * head budgets hurt).  Among equal scores the lower flat index is kept first,
  * which makes the mask unique.
  *
- *   scores    [N] float32, finite and >= 0 (NaN/Inf give an unspecified but
- *             in-bounds result).
+ *   scores    [N] float32, >= 0, compared by value: -0.0 equals 0.0 and
+ *             +inf ranks above every finite score.  Negative or NaN scores
+ *             give an unspecified result that still keeps exactly k and stays
+ *             in bounds.
  *   k         0..N (use kvzip_keep_count for a ratio).
  *   n_heads   >= 1, N % n_heads == 0.
  *   keep      [N] uint8 out: 1 = kept.  Any alignment.
  *   offsets   [n_heads + 1] int64 out: offsets[h] = kept rows in heads < h;
  *             offsets[n_heads] = k.  8-byte aligned.
- *   threshold float out or NULL: the k-th largest score (+inf if k == 0).
+ *   threshold float out or NULL: the k-th largest score, as a non-negative
+ *             value (+inf if k == 0).
  *   N < 2^31.
  *   workspace >= kvzip_select_workspace_size(N, n_heads) bytes, 256-byte
  *             aligned.  Its first 4 bytes are a sticky status word, as in the
