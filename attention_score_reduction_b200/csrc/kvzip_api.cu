@@ -90,7 +90,7 @@ size_t kvzip_score_workspace_size(int B, int G, int n_in) {
 static kvzip_status score_passes(int passes, int sum_agg, kvzip_dtype dt, const void* q, const void* k_ctx,
                                  const void* k_self, float* scores, int B, int G, int n_in,
                                  int n_c, int d, float scale, void* workspace, size_t ws_bytes,
-                                 void* stream) {
+                                 void* stream, unsigned int* score_hist = nullptr) {
   if (dt != KVZIP_BF16 && dt != KVZIP_F32) return KVZIP_ERR_INVALID_ARG;
   if (B < 0 || G < 0 || n_in < 0 || n_c < 0) return KVZIP_ERR_INVALID_ARG;
   if (d != 128 && d != 256) return d > 0 ? KVZIP_ERR_UNSUPPORTED : KVZIP_ERR_INVALID_ARG;
@@ -122,6 +122,7 @@ static kvzip_status score_passes(int passes, int sum_agg, kvzip_dtype dt, const 
   a.timeout_ns = g_timeout_ns.load();
   a.passes = passes;
   a.sum_aggregation = sum_agg;
+  a.score_hist = score_hist;
   a.test_stall = g_test_stall.load();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int launches = 0;
@@ -153,6 +154,15 @@ kvzip_status kvzip_score_colmax(kvzip_dtype dt, const void* q, const void* k_ctx
                                 void* stream) {
   return score_passes(2, 0, dt, q, k_ctx, k_self, scores, B, G, n_in, n_c, d, scale, workspace,
                       ws_bytes, stream);
+}
+
+kvzip_status kvzip_score_colmax_hist(kvzip_dtype dt, const void* q, const void* k_ctx,
+                                     const void* k_self, float* scores, int B, int G, int n_in,
+                                     int n_c, int d, float scale, unsigned int* score_hist,
+                                     void* workspace, size_t ws_bytes, void* stream) {
+  if (!score_hist || !aligned(score_hist, 4)) return KVZIP_ERR_INVALID_ARG;
+  return score_passes(2, 0, dt, q, k_ctx, k_self, scores, B, G, n_in, n_c, d, scale, workspace,
+                      ws_bytes, stream, score_hist);
 }
 
 kvzip_status kvzip_score_chunk_sum(const void* q, const void* k_ctx, const void* k_self,
@@ -199,7 +209,8 @@ kvzip_status kvzip_workspace_status(void* workspace, void* stream) {
   const uint32_t zero = 0;
   if (cudaMemcpy(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
     return KVZIP_ERR_CUDA;
-  return (word & kvzip::kStatusTimeout) ? KVZIP_ERR_TIMEOUT : KVZIP_OK;
+  if (word & kvzip::kStatusTimeout) return KVZIP_ERR_TIMEOUT;
+  return (word & kvzip::kStatusHistMismatch) ? KVZIP_ERR_INVALID_ARG : KVZIP_OK;
 }
 
 int64_t kvzip_keep_count(double r, int64_t N) {
@@ -212,9 +223,10 @@ size_t kvzip_select_workspace_size(int64_t N, int64_t n_heads) {
   return kvzip::select_fused_ws_bytes(N, n_heads);
 }
 
-kvzip_status kvzip_select(const float* scores, int64_t N, int64_t k, int64_t n_heads,
-                          uint8_t* keep, int64_t* offsets, float* threshold, void* workspace,
-                          size_t ws_bytes, void* stream) {
+static kvzip_status select_impl(const float* scores, int64_t N, int64_t k, int64_t n_heads,
+                                const unsigned int* score_hist, uint8_t* keep, int64_t* offsets,
+                                float* threshold, void* workspace, size_t ws_bytes,
+                                void* stream) {
   if (N < 0 || n_heads <= 0 || k < 0 || k > N) return KVZIP_ERR_INVALID_ARG;
   if (N % n_heads != 0 || N >= (int64_t{1} << 31) || n_heads > (int64_t{1} << 24))
     return KVZIP_ERR_INVALID_ARG;
@@ -241,11 +253,28 @@ kvzip_status kvzip_select(const float* scores, int64_t N, int64_t k, int64_t n_h
   a.threshold = threshold;
   a.ws = workspace;
   a.ws_bytes = ws_bytes;
+  a.hist_in = score_hist;
   int launches = 0;
   cudaError_t e =
       kvzip::launch_select_fused(a, g_timeout_ns.load(), g_test_stall.load(), s, &launches);
   if (e == cudaSuccess) g_last_launches.store(launches);
   return from_cuda(e);
+}
+
+kvzip_status kvzip_select(const float* scores, int64_t N, int64_t k, int64_t n_heads,
+                          uint8_t* keep, int64_t* offsets, float* threshold, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  return select_impl(scores, N, k, n_heads, nullptr, keep, offsets, threshold, workspace,
+                     ws_bytes, stream);
+}
+
+kvzip_status kvzip_select_hist(const float* scores, int64_t N, int64_t k, int64_t n_heads,
+                               const unsigned int* score_hist, uint8_t* keep, int64_t* offsets,
+                               float* threshold, void* workspace, size_t ws_bytes,
+                               void* stream) {
+  if (!score_hist || !aligned(score_hist, 4)) return KVZIP_ERR_INVALID_ARG;
+  return select_impl(scores, N, k, n_heads, score_hist, keep, offsets, threshold, workspace,
+                     ws_bytes, stream);
 }
 
 int kvzip_select_shard_bins(int round) { return kvzip::shard_bins(round); }

@@ -9,6 +9,7 @@ namespace kvzip {
 
 // Status bits the kernels OR into the workspace header word.
 constexpr uint32_t kStatusTimeout = 1u;
+constexpr uint32_t kStatusHistMismatch = 2u;   // kvzip_select_hist: histogram != scores
 
 // Bytes reserved at the front of the scoring workspace for the status word.
 constexpr size_t kScoreWsHeader = 256;
@@ -33,6 +34,8 @@ struct ScoreArgs {
   int passes;         // bit 0: pass 1 (row log-sum-exp), bit 1: pass 2 (column max)
   int test_stall;     // tensor-core scorer only: loader issues nothing (timeout tests)
   int sum_aggregation = 0;  // pass 2 adds column sums instead of taking maxima
+  uint32_t* score_hist = nullptr;  // pass 2 (maxima): each resulting score counted in its
+                                   // round-1 bin (kScoreHistBins bins, see score_hist_add)
 };
 
 // Tensor-core (tcgen05) scorer for bf16 inputs.  Returns a cudaError_t.
@@ -48,6 +51,7 @@ struct SelectArgs {
   float* threshold;
   void* ws;
   size_t ws_bytes;
+  const uint32_t* hist_in = nullptr;   // round-1 histogram of the scores, or null
 };
 // One cooperative launch, two reads of the scores (kvzip_select).
 size_t select_fused_ws_bytes(int64_t N, int64_t n_heads);
@@ -161,5 +165,18 @@ cudaError_t bounds_flag_decode(unsigned int* out);
 // order, and -0.0 ranks as 0.0 (its raw bits would rank above every score).
 // Every kernel that compares or orders score bits reads them through mag.
 __host__ __device__ __forceinline__ uint32_t mag(uint32_t w) { return w & 0x7FFFFFFFu; }
+
+// Round-1 histogram of the selection: bin = the top 13 bits of mag(bits).
+constexpr int kScoreHistBins = 8192;
+constexpr int kScoreHistShift = 19;
+
+// Count score v in its round-1 bin.  Lanes of the calling warp that are here
+// together and share a bin add once (scores cluster in a few hundred bins).
+__device__ __forceinline__ void score_hist_add(uint32_t* hist, float v) {
+  const uint32_t bin = mag(__float_as_uint(v)) >> kScoreHistShift;
+  const uint32_t peers = __match_any_sync(__activemask(), bin);
+  if ((threadIdx.x & 31u) == static_cast<uint32_t>(__ffs(peers) - 1))
+    atomicAdd(hist + bin, static_cast<uint32_t>(__popc(peers)));
+}
 
 }  // namespace kvzip

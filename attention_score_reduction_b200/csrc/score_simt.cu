@@ -30,6 +30,7 @@ struct SimtParams {
   float* lse2;
   int n_in, n_c, d, R, R_pad;
   float c;
+  uint32_t* hist;       // null, or the round-1 histogram of the new scores (pass 2)
 };
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -163,7 +164,10 @@ __global__ void __launch_bounds__(kSimtThreads)
       if (lane == r) br = best[r];
     if (key < p.n_c) {
       float* dst = p.scores + static_cast<size_t>(b) * p.n_c + key;
-      *dst = fmaxf(*dst, exp2f(br));
+      const float s_new = fmaxf(*dst, exp2f(br));
+      *dst = s_new;
+      if (p.hist)
+        atomicAdd(p.hist + (mag(__float_as_uint(s_new)) >> kScoreHistShift), 1u);
     }
   }
 }
@@ -181,6 +185,7 @@ cudaError_t launch_score_simt_f32(const ScoreArgs& a, cudaStream_t s, int* launc
   p.R = a.R;
   p.R_pad = a.R_pad;
   p.c = a.scale * 1.4426950408889634f;
+  p.hist = a.score_hist;
   const size_t smem = 2 * kSimtRows * (a.d + 1) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(simt_lse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));

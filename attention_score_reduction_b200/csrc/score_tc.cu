@@ -138,6 +138,7 @@ struct TcParams {
   float c;            // scale * log2(e)
   uint64_t timeout_ns;
   int test_stall;     // test hook: the loader issues no copies, so every wait runs out
+  uint32_t* hist;     // pass 2 (maxima) only, or null: round-1 histogram of the new scores
 };
 
 // SUM (pass 2 only): column sums of the probabilities instead of maxima (the
@@ -475,10 +476,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_barrier_sync(1 + t, 2 * kBM);
         if (par == 0 && !*abort_flag && arow < p.n_c && in_bounds(b < static_cast<int>(gridDim.y))) {
           float* dst = p.scores + static_cast<size_t>(b) * p.n_c + arow;
-          if (SUM)
+          if (SUM) {
             *dst += best + xchg->x;
-          else
-            *dst = fmaxf(*dst, ex2_approx(fmaxf(best, xchg->x)));
+          } else {
+            const float s_new = fmaxf(*dst, ex2_approx(fmaxf(best, xchg->x)));
+            *dst = s_new;
+            if (p.hist) score_hist_add(p.hist, s_new);
+          }
         }
       }
     } else if (!PASS2 && par == 0) {
@@ -535,6 +539,7 @@ static cudaError_t launch_tc(const ScoreArgs& a, cudaStream_t s, int* launches) 
   p.c = a.scale * 1.4426950408889634f;
   p.timeout_ns = a.timeout_ns;
   p.test_stall = a.test_stall;
+  p.hist = nullptr;
 
   // Maps of box height BN (per pass).  With A in shared memory (BN = kBM) a map
   // of the A operand serves the A tiles; with A in TMEM its rows are copied from
@@ -558,6 +563,7 @@ static cudaError_t launch_tc(const ScoreArgs& a, cudaStream_t s, int* launches) 
       !make_map(&qmap2, a.q, a.B, a.R, D, L2::BN))
     return cudaErrorInvalidValue;
   p.a_ptr = static_cast<const uint16_t*>(a.k_ctx);
+  p.hist = a.sum_aggregation ? nullptr : a.score_hist;
   dim3 g2((a.n_c + kATiles * kBM - 1) / (kATiles * kBM), a.B);
   if (a.sum_aggregation)
     score_tc_kernel<D, true, true><<<g2, kThreads, L2::SMEM_ALLOC, s>>>(qmap2, qmap2, kmap2, p);

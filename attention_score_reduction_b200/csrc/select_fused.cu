@@ -69,7 +69,8 @@ constexpr size_t kLine = 128;             // one counter per 128-byte line
 constexpr size_t kOffH1 = kOffSync + (kBarGroups + 2) * kLine;
 constexpr size_t kOffH2 = kOffH1 + kBins1 * 4;
 constexpr size_t kOffH3 = kOffH2 + kBins2 * 4;
-constexpr size_t kOffHeads = kOffH3 + kBins3 * 4;
+constexpr size_t kOffKeptC = kOffH3 + kBins3 * 4;   // scores the mask pass keeps (one word)
+constexpr size_t kOffHeads = kOffKeptC + 256;
 
 __host__ __device__ size_t up256(size_t x) { return (x + 255) / 256 * 256; }
 
@@ -112,6 +113,7 @@ struct Params {
   int vec;               // scores 16-byte aligned: 16-byte loads
   int vec_keep;          // keep 4-byte aligned: 4-byte mask stores
   int test_stall;        // test hook: block 0 never reaches a barrier, so the others time out
+  const uint32_t* hist_in;   // round-1 histogram of the scores (phase A is skipped), or null
 };
 
 // Grid-barrier words, each on its own 128-byte line: kBarGroups first-level
@@ -316,14 +318,14 @@ struct Round1 {
 // (flat index, mag bits) pairs to seg in flat order (positions from one warp
 // scan of per-load counts packed in bytes; each lane then walks its own
 // candidate bits), their round-2 digits histogrammed into h2, and each step's
-// kept scores passed to cnt.add_step.  Each group of four scores gets its
+// kept scores passed to cnt.add_step and added to *kept.  Each group of four scores gets its
 // decisions as byte masks: on the fast path four float subtractions and the
 // sign bytes of their results, otherwise integer compares.  Returns the
 // warp's candidate count.
 template <class Counter>
 __device__ uint32_t mask_pass(const float* __restrict__ s, uint32_t wl, uint32_t wh,
                               const Round1 r1, bool vec, bool vec_keep, uint8_t* keep,
-                              uint2* seg, uint32_t* h2, Counter& cnt) {
+                              uint2* seg, uint32_t* h2, Counter& cnt, uint32_t* kept) {
   const uint4* s4 = reinterpret_cast<const uint4*>(s);
   const uint32_t* su = reinterpret_cast<const uint32_t*>(s);
   const uint32_t lane = threadIdx.x & 31;
@@ -397,7 +399,9 @@ __device__ uint32_t mask_pass(const float* __restrict__ s, uint32_t wl, uint32_t
       cw[q] = c;
       any |= c;
     }
-    cnt.add_step(g0, min(g0 + kWarpStep, wh), ib, kws, (kacc * 0x01010101u) >> 24);
+    const uint32_t n_kept = (kacc * 0x01010101u) >> 24;
+    *kept += n_kept;
+    cnt.add_step(g0, min(g0 + kWarpStep, wh), ib, kws, n_kept);
     if (__any_sync(0xffffffffu, any != 0)) {
       // candidates per load, one byte each; <= 128 per warp, so the scan's bytes never carry
       const uint32_t packed = __popc(cw[0]) | (__popc(cw[1]) << 8) | (__popc(cw[2]) << 16) |
@@ -464,7 +468,10 @@ __device__ void pick_bin(const uint32_t* h, uint64_t k_rem, int* bin_out, uint64
     if (lane >= o) inc += n;
   }
   if (lane == 31) wsum[warp] = inc;
-  if (threadIdx.x == 0) bin_s = -1;
+  if (threadIdx.x == 0) {
+    bin_s = -1;   // k_rem beyond the histogram's total
+    above_s = 0;
+  }
   __syncthreads();
   unsigned long long base = 0;
   for (int w = 0; w < warp; ++w) base += wsum[w];
@@ -567,8 +574,12 @@ __global__ void __launch_bounds__(kThr, 2)
   if (p.test_stall && blockIdx.x == 0) return;
   for (int i = threadIdx.x; i < kHeadWin; i += kThr) win[i] = 0;
 
+  // With a given round-1 histogram the first read and its barrier are skipped;
+  // the histogram is checked against the scores after the mask pass.
+  const bool given = p.hist_in != nullptr && !none;
+
   // ------------------------------------------------------------ A: round-1 histogram
-  if (!none) {
+  if (!none && !given) {
     for (int i = threadIdx.x; i < kBins1; i += kThr) h1[i] = 0;
     __syncthreads();
     hist_top(p.s, lo, hi, p.vec != 0, h1);
@@ -576,15 +587,14 @@ __global__ void __launch_bounds__(kThr, 2)
     for (int i = threadIdx.x; i < kBins1; i += kThr)
       if (h1[i]) atomicAdd(g1 + i, h1[i]);
   }
-  if (!grid_barrier(sy, status, p.timeout_ns)) return;
+  if (!given && !grid_barrier(sy, status, p.timeout_ns)) return;
 
   // ------------------------------------------------------------ B: bin of round 1
   int b1 = -1;
-  uint64_t k_rem = p.k;
+  uint64_t k_rem = p.k, above1 = 0;
   if (!none) {
-    uint64_t above;
-    pick_bin<kBins1>(g1, k_rem, &b1, &above);
-    k_rem -= above;
+    pick_bin<kBins1>(given ? p.hist_in : g1, k_rem, &b1, &above1);
+    k_rem -= above1;
   }
 
   // ------------------------------------------------------------ C: mask, candidates, round-2 histogram
@@ -592,18 +602,41 @@ __global__ void __launch_bounds__(kThr, 2)
   __syncthreads();
   const uint32_t ub1 = static_cast<uint32_t>(b1);
   HeadCounter hc(lo / p.n_c, p.n_c, p.n_heads, win, heads);
+  uint32_t kept_c = 0;
   const uint32_t n_w = mask_pass(p.s, wl, wh, Round1(b1, none), p.vec != 0, p.vec_keep != 0,
-                                 p.keep, wseg, h2, hc);
+                                 p.keep, wseg, h2, hc, &kept_c);
   hc.flush();
+  if (given) {   // scores this block kept in the mask pass
+    uint32_t tot;
+    block_excl(kept_c, tmp, &tot);
+    if (threadIdx.x == 0 && tot) atomicAdd(reinterpret_cast<uint32_t*>(p.ws + kOffKeptC), tot);
+  }
   __syncthreads();
   for (int i = threadIdx.x; i < kBins2; i += kThr)
     if (h2[i]) atomicAdd(g2 + i, h2[i]);
   if (!grid_barrier(sy, status, p.timeout_ns)) return;
 
+  // A given histogram must agree with the scores above and inside bin b1; if it
+  // does, b1 and k_rem are what phase A would have found.  Otherwise nothing is
+  // kept: every block clears its mask bytes and block 0 writes empty offsets.
+  bool mismatch = false;
+  if (given) {
+    uint32_t c = 0, tot;
+    for (int i = threadIdx.x; i < kBins2; i += kThr) c += __ldcg(g2 + i);
+    block_excl(c, tmp, &tot);
+    const uint32_t kept_tot = __ldcg(reinterpret_cast<const uint32_t*>(p.ws + kOffKeptC));
+    // (a histogram with fewer than k scores has no bin b1 at all)
+    mismatch = b1 < 0 || tot != __ldcg(p.hist_in + b1) || kept_tot != above1;
+    if (mismatch) {
+      if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(status, kStatusHistMismatch);
+      for (uint32_t f = lo + threadIdx.x; f < hi; f += kThr) p.keep[f] = 0;
+    }
+  }
+
   uint32_t tau = 0x7F800000u;
   uint64_t take_eq = 0;
   bool rank_ties = false;
-  if (!none) {
+  if (!none && !mismatch) {
     // ---------------------------------------------------------- D: round 2, round-3 histogram
     int b2;
     uint64_t above;
@@ -690,7 +723,7 @@ __global__ void __launch_bounds__(kThr, 2)
   unsigned long long carry = 0;
   for (uint32_t base = 0; base < p.n_heads; base += kThr) {
     const uint32_t hh = base + threadIdx.x;
-    const uint32_t c = hh < p.n_heads ? __ldcg(heads + hh) : 0u;
+    const uint32_t c = hh < p.n_heads && !mismatch ? __ldcg(heads + hh) : 0u;
     uint32_t tot;
     const uint32_t ex = block_excl(c, tmp, &tot);
     if (hh < p.n_heads) p.offsets[hh] = static_cast<int64_t>(carry + ex);
@@ -698,7 +731,7 @@ __global__ void __launch_bounds__(kThr, 2)
   }
   if (threadIdx.x == 0) {
     p.offsets[p.n_heads] = static_cast<int64_t>(carry);
-    if (p.threshold) *p.threshold = none ? INFINITY : __uint_as_float(tau);
+    if (p.threshold) *p.threshold = none || mismatch ? INFINITY : __uint_as_float(tau);
   }
 }
 
@@ -748,7 +781,9 @@ __global__ void __launch_bounds__(kThr, 2)
   for (int i = threadIdx.x; i < kBins2; i += kThr) h2[i] = 0;
   __syncthreads();
   NoCounter nc;
-  const uint32_t n_w = mask_pass(sh, wl, wh, Round1(b1, none), v4, k4, kh, wseg, h2, nc);
+  uint32_t kept_unused = 0;
+  const uint32_t n_w =
+      mask_pass(sh, wl, wh, Round1(b1, none), v4, k4, kh, wseg, h2, nc, &kept_unused);
   __syncthreads();
   if (none) return;
   int b2;
@@ -871,6 +906,7 @@ cudaError_t launch_select_fused(const SelectArgs& a, uint64_t timeout_ns, int te
   p.vec = reinterpret_cast<uintptr_t>(a.scores) % 16 == 0 ? 1 : 0;   // ranges start on 4 scores
   p.vec_keep = reinterpret_cast<uintptr_t>(a.keep) % 4 == 0 ? 1 : 0;
   p.test_stall = test_stall;
+  p.hist_in = a.hist_in;
   void* args[] = {&p};
   e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(select_fused_kernel),
                                   dim3(P_used), dim3(kThr), args, 0, s);

@@ -40,6 +40,8 @@ def _load() -> ctypes.CDLL:
         "kvzip_score_chunk": (i32, [i32, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, sz, vp]),
         "kvzip_score_lse": (i32, [i32, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, sz, vp]),
         "kvzip_score_colmax": (i32, [i32, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, sz, vp]),
+        "kvzip_score_colmax_hist": (i32, [i32, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp,
+                                          sz, vp]),
         "kvzip_score_context_workspace_size": (sz, [i32, i32, i32]),
         "kvzip_score_context": (i32, [i32, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, vp,
                                       sz, vp]),
@@ -50,6 +52,7 @@ def _load() -> ctypes.CDLL:
         "kvzip_keep_count": (i64, [f64, i64]),
         "kvzip_select_workspace_size": (sz, [i64, i64]),
         "kvzip_select": (i32, [vp, i64, i64, i64, vp, vp, vp, vp, sz, vp]),
+        "kvzip_select_hist": (i32, [vp, i64, i64, i64, vp, vp, vp, vp, vp, sz, vp]),
         "kvzip_select_noalloc": (i32, [vp, i64, i64, i64, vp, vp, vp, vp]),
         "kvzip_select_shard_bins": (i32, [i32]),
         "kvzip_select_shard_workspace_size": (sz, [i64, i64]),
@@ -135,15 +138,35 @@ def new_score_workspace(B: int, G: int, n_in: int, device=None) -> torch.Tensor:
     return torch.zeros(max(n, 256), dtype=torch.uint8, device=device or "cuda")
 
 
+SCORE_HIST_BINS = 8192   # KVZIP_SCORE_HIST_BINS
+
+
+def new_score_hist(device=None) -> torch.Tensor:
+    """A zeroed round-1 histogram for score_chunk(..., hist=) / select(..., hist=)."""
+    return torch.zeros(SCORE_HIST_BINS, dtype=torch.int32, device=device or "cuda")
+
+
 def score_chunk(q: torch.Tensor, k_ctx: torch.Tensor, k_self: torch.Tensor, scores: torch.Tensor,
                 workspace: torch.Tensor | None = None, scale: float = 0.0, stream=None,
-                which: str = "both"):
+                which: str = "both", hist: torch.Tensor | None = None):
     """scores[b][j] = max(scores[b][j], max_rho softmax(...)[rho][j]) for one chunk.
 
     q [B][G][n_in][d], k_ctx [B][n_c][d], k_self [B][n_in][d] (bf16 or fp32,
     same dtype), scores [B][n_c] float32.  ``which`` = "both" (kvzip_score_chunk),
-    "lse" (kvzip_score_lse) or "colmax" (kvzip_score_colmax).
+    "lse" (kvzip_score_lse) or "colmax" (kvzip_score_colmax).  With ``hist``
+    (int32 [SCORE_HIST_BINS], zeroed) the column-max half is
+    kvzip_score_colmax_hist: the resulting scores are counted in their
+    round-1 bins.
     """
+    if hist is not None:
+        _dev_contig("hist", hist, torch.int32)
+        if hist.numel() != SCORE_HIST_BINS:
+            raise ValueError("hist must hold SCORE_HIST_BINS counts")
+        if which == "both":
+            score_chunk(q, k_ctx, k_self, scores, workspace, scale, stream, "lse")
+            return score_chunk(q, k_ctx, k_self, scores, workspace, scale, stream, "colmax", hist)
+        if which != "colmax":
+            raise ValueError("hist goes with the column-max half")
     fn = {"both": _lib.kvzip_score_chunk, "lse": _lib.kvzip_score_lse,
           "colmax": _lib.kvzip_score_colmax}[which]
     for n, t in (("q", q), ("k_ctx", k_ctx), ("k_self", k_self)):
@@ -155,6 +178,13 @@ def score_chunk(q: torch.Tensor, k_ctx: torch.Tensor, k_self: torch.Tensor, scor
         raise ValueError("shape mismatch between q, k_ctx, k_self and scores")
     if workspace is None:
         workspace = new_score_workspace(B, G, n_in, q.device)
+    if hist is not None:
+        s = _lib.kvzip_score_colmax_hist(
+            _dtype_code(q), _ptr(q), _ptr(k_ctx), _ptr(k_self), _ptr(scores), B, G, n_in, n_c, d,
+            float(scale), _ptr(hist), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream(stream))
+        _check(s, "kvzip_score_colmax_hist")
+        return scores
     s = fn(_dtype_code(q), _ptr(q), _ptr(k_ctx), _ptr(k_self), _ptr(scores), B, G, n_in, n_c, d,
            float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(),
            _stream(stream))
@@ -257,9 +287,11 @@ def select_workspace_size(N: int, n_heads: int) -> int:
 
 def select(scores: torch.Tensor, k: int, n_heads: int, keep: torch.Tensor | None = None,
            offsets: torch.Tensor | None = None, threshold: torch.Tensor | None = None,
-           workspace: torch.Tensor | None = None, stream=None):
+           workspace: torch.Tensor | None = None, stream=None, hist: torch.Tensor | None = None):
     """Global top-k keep mask, per-head offsets and the threshold score.
 
+    With ``hist`` (the scores' round-1 histogram, as score_chunk(..., hist=)
+    leaves it) this is kvzip_select_hist, which reads the scores once.
     Returns (keep uint8 [N], offsets int64 [n_heads+1], threshold float32 [1]).
     """
     _dev_contig("scores", scores, torch.float32)
@@ -271,6 +303,15 @@ def select(scores: torch.Tensor, k: int, n_heads: int, keep: torch.Tensor | None
     if workspace is None:
         workspace = torch.zeros(max(select_workspace_size(N, n_heads), 256), dtype=torch.uint8,
                                 device=dev)
+    if hist is not None:
+        _dev_contig("hist", hist, torch.int32)
+        if hist.numel() != SCORE_HIST_BINS:
+            raise ValueError("hist must hold SCORE_HIST_BINS counts")
+        s = _lib.kvzip_select_hist(_ptr(scores), N, int(k), int(n_heads), _ptr(hist), _ptr(keep),
+                                   _ptr(offsets), _ptr(threshold), _ptr(workspace),
+                                   workspace.numel(), _stream(stream))
+        _check(s, "kvzip_select_hist")
+        return keep, offsets, threshold
     s = _lib.kvzip_select(_ptr(scores), N, int(k), int(n_heads), _ptr(keep), _ptr(offsets),
                           _ptr(threshold), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(s, "kvzip_select")

@@ -4,11 +4,16 @@ selection and per-head compaction, through libkvzip.
 This is the user-facing call.  ``Compressor`` owns the device buffers for one
 context shape and runs the three C-ABI calls on a CUDA stream:
 
-  1. ``kvzip_score_context`` (all chunks) or ``kvzip_score_chunk`` once per
-     reconstruction chunk (blog post section 4.5: chunked scoring keeps memory
-     linear in n_c), merging into the L x H x n_c score tensor by a running max;
-  2. ``kvzip_select`` once per context (scime.ai summary, "Approach": evict the
-     lowest-scoring pairs once, query-agnostically), global over (l, h, j);
+  1. ``kvzip_score_context`` (all chunks but the last) or ``kvzip_score_chunk``
+     once per reconstruction chunk (blog post section 4.5: chunked scoring
+     keeps memory linear in n_c), merging into the L x H x n_c score tensor by
+     a running max.  The last chunk's column-max half is
+     ``kvzip_score_colmax_hist``: it also counts the final scores in the
+     selection's round-1 histogram;
+  2. ``kvzip_select_hist`` once per context (scime.ai summary, "Approach":
+     evict the lowest-scoring pairs once, query-agnostically), global over
+     (l, h, j), reading the scores once; with several ranks, the sharded
+     selection;
   3. ``kvzip_compact`` once, packing the kept K/V rows per head.
 
 ``compress_from_host`` is the same path for inputs that start in (pinned)
@@ -66,13 +71,29 @@ class Compressor:
         self.keep = torch.empty(N, dtype=torch.uint8, device=self.device)
         self.offsets = torch.empty(units + 1, dtype=torch.int64, device=self.device)
         self.threshold = torch.empty(1, dtype=torch.float32, device=self.device)
+        # round-1 histogram of the final scores, counted by the last chunk's
+        # column-max pass; the one-GPU selection then reads the scores once
+        self.score_hist = kz.new_score_hist(self.device) if group is None else None
+        self.hist_ready = False
         self.launches = 0
 
     def reset(self):
         self.scores.zero_()
+        if self.score_hist is not None:
+            self.score_hist.zero_()
+        self.hist_ready = False
 
-    def score_chunk(self, q, k_ctx, k_self, scale: float = 0.0, stream=None):
-        kz.score_chunk(q, k_ctx, k_self, self.scores, self.score_ws, scale, stream)
+    def score_chunk(self, q, k_ctx, k_self, scale: float = 0.0, stream=None, last: bool = False):
+        """One chunk; ``last`` (the context's final chunk) also counts the
+        final scores in the selection's round-1 histogram."""
+        if last and self.score_hist is not None:
+            kz.score_chunk(q, k_ctx, k_self, self.scores, self.score_ws, scale, stream, "lse")
+            self.launches += kz.last_launch_count()
+            kz.score_chunk(q, k_ctx, k_self, self.scores, self.score_ws, scale, stream, "colmax",
+                           hist=self.score_hist)
+            self.hist_ready = True
+        else:
+            kz.score_chunk(q, k_ctx, k_self, self.scores, self.score_ws, scale, stream)
         self.launches += kz.last_launch_count()
 
     def keep_capacity(self, r: float) -> int:
@@ -87,7 +108,8 @@ class Compressor:
         if self.group is None:
             kept = kz.keep_count(r, self.scores.numel())
             kz.select(self.scores.view(-1), kept, self.units, self.keep, self.offsets,
-                      self.threshold, self.select_ws, stream)
+                      self.threshold, self.select_ws, stream,
+                      hist=self.score_hist if self.hist_ready else None)
             self.launches += kz.last_launch_count()
             return kept
         from . import sharded
@@ -109,8 +131,13 @@ class Compressor:
         """k_ctx, v: [units][n_c][d] bf16 on the device; chunks: iterable of
         (q [units][G][n_in][d], k_self [units][n_in][d]) device tensors."""
         self.reset()
-        kz.score_context(list(chunks), k_ctx, self.scores, self.score_ws, scale, stream)
-        self.launches += kz.last_launch_count()
+        chunks = list(chunks)
+        if len(chunks) > 1:
+            kz.score_context(chunks[:-1], k_ctx, self.scores, self.score_ws, scale, stream)
+            self.launches += kz.last_launch_count()
+        if chunks:
+            q_last, ks_last = chunks[-1]
+            self.score_chunk(q_last, k_ctx, ks_last, scale=scale, stream=stream, last=True)
         kept = self.select(r, stream)
         k_out, v_out, pos = self.compact(k_ctx, v, kept, *(out or (None, None, None)),
                                          stream=stream)
@@ -171,7 +198,7 @@ def compress_from_host(comp: Compressor, k_ctx_h, v_h, q_chunks_h, ks_chunks_h, 
             up = torch.cuda.Event()
             up.record(copy)
         main.wait_event(up)
-        comp.score_chunk(qd, dev_bufs["k_ctx"], ksd, scale)
+        comp.score_chunk(qd, dev_bufs["k_ctx"], ksd, scale, last=c == len(q_chunks_h) - 1)
         done = torch.cuda.Event()
         done.record(main)
         freed[slot] = done

@@ -210,7 +210,6 @@ def run_only(args):
     r = args.r if args.r is not None else wl.r[0]
     peaks = bu.load_peaks(os.path.join(ROOT, "MEASURED_PEAKS.json"))
     N = wl.units * wl.n_c
-    times = []
     if args.only == "select":
         s = synth.random_scores(wl.units, wl.n_c, seed=11, device=dev).reshape(-1)
         k = kz.keep_count(r, N)
@@ -219,6 +218,11 @@ def run_only(args):
         thr = torch.empty(1, dtype=torch.float32, device=dev)
         ws = torch.zeros(kz.select_workspace_size(N, wl.units), dtype=torch.uint8, device=dev)
         fn = lambda: kz.select(s, k, wl.units, keep, off, thr, ws)  # noqa: E731
+        # the scores' round-1 histogram, as the last chunk's column-max pass would
+        # leave it (counted here with torch outside the timed calls)
+        hist = torch.bincount((s.view(torch.int32) & 0x7FFFFFFF) >> 19,
+                              minlength=kz.SCORE_HIST_BINS).to(torch.int32)
+        fn_hist = lambda: kz.select(s, k, wl.units, keep, off, thr, ws, hist=hist)  # noqa: E731
         nbytes = N * 4 + N
     else:
         units = wl.H      # one layer
@@ -232,20 +236,28 @@ def run_only(args):
         fn = lambda: kz.compact(k_c, v, keep, off, kept, k_out, v_out, pos)  # noqa: E731
         nbytes = s.numel() + kept * wl.d * 2 * 2 * 2 + kept * 4
     flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
-    for i in range(args.warmup + args.steps):
-        flush.fill_(i & 0xff)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        fn()
-        e1.record()
-        torch.cuda.synchronize()
-        if i >= args.warmup:
-            times.append(e0.elapsed_time(e1))
-    ms = sum(times) / len(times)
-    gbs = nbytes / (ms * 1e-3) / 1e9
-    print(json.dumps({"kernel": args.only, "workload": wl.name, "ms": ms, "bytes": nbytes,
-                      "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
-                      "peak_source": peaks["source"], "l2": "flushed before each launch"}))
+
+    def timed(f):
+        times = []
+        for i in range(args.warmup + args.steps):
+            flush.fill_(i & 0xff)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            f()
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                times.append(e0.elapsed_time(e1))
+        ms = sum(times) / len(times)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return {"ms": ms, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"]}
+
+    out = {"kernel": args.only, "workload": wl.name, "bytes": nbytes}
+    out.update(timed(fn))
+    if args.only == "select":   # kvzip_select_hist: the first read replaced by the histogram
+        out["given_hist"] = timed(fn_hist)
+    out.update({"peak_source": peaks["source"], "l2": "flushed before each launch"})
+    print(json.dumps(out))
 
 
 def main():
@@ -306,7 +318,10 @@ def main():
                 if timed:
                     e0, e1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
                     e0.record(stream)
-                kz.score_chunk(q, k_ctx, ks, comp.scores, comp.score_ws, which=which)
+                last = which == "colmax" and c == wl.n_chunks - 1 and comp.score_hist is not None
+                kz.score_chunk(q, k_ctx, ks, comp.scores, comp.score_ws, which=which,
+                               hist=comp.score_hist if last else None)
+                comp.hist_ready = comp.hist_ready or last
                 launches += kz.last_launch_count()
                 if timed:
                     e1.record(stream)

@@ -111,6 +111,23 @@ kvzip_status kvzip_score_colmax(kvzip_dtype dt, const void* q, const void* k_ctx
                                 void* stream);
 
 /*
+ * kvzip_score_colmax that also counts every score it leaves in `scores` in
+ * the selection's first radix round: score_hist[b] += the number of those
+ * scores whose |s| bits, shifted right by 19 (the top 13 bits), equal b.
+ * Called for a context's last chunk, score_hist is then the round-1
+ * histogram of the final scores, and kvzip_select_hist skips its own first
+ * read of them.  score_hist: KVZIP_SCORE_HIST_BINS uint32 on the device,
+ * zeroed by the caller before the call; other arguments as kvzip_score_colmax.
+ * The pages have no counterpart: it fuses work of the selection into the
+ * kernel that writes the scores.
+ */
+#define KVZIP_SCORE_HIST_BINS 8192
+kvzip_status kvzip_score_colmax_hist(kvzip_dtype dt, const void* q, const void* k_ctx,
+                                     const void* k_self, float* scores, int B, int G, int n_in,
+                                     int n_c, int d, float scale, unsigned int* score_hist,
+                                     void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Multi-chunk scoring: all reconstruction chunks of one context in one call
  * (blog post section 4.5: the context is reconstructed chunk by chunk and
  * the chunk scores are merged by a running maximum).  Equivalent to
@@ -146,9 +163,11 @@ kvzip_status kvzip_score_context(kvzip_dtype dt, int n_chunks, const void* const
  * call on the same workspace overwrites it.  Host-only, no CUDA call. */
 kvzip_status kvzip_score_lse_layout(int G, int n_in, size_t* offset_bytes, int64_t* row_stride);
 
-/* Synchronise `stream`, then report (and clear) the status word the scoring
- * kernels leave in `workspace`: KVZIP_OK, or KVZIP_ERR_TIMEOUT when a kernel
- * abandoned a pipeline wait (its scores for that call are then incomplete). */
+/* Synchronise `stream`, then report (and clear) the status word the kernels
+ * leave in `workspace`: KVZIP_OK; KVZIP_ERR_TIMEOUT when a kernel abandoned a
+ * pipeline or grid wait (its results for that call are then incomplete); or
+ * KVZIP_ERR_INVALID_ARG when kvzip_select_hist found that its histogram does
+ * not match the scores. */
 kvzip_status kvzip_workspace_status(void* workspace, void* stream);
 
 /* Longest a scoring kernel waits on one pipeline stage before it gives up,
@@ -208,6 +227,21 @@ size_t kvzip_select_workspace_size(int64_t N, int64_t n_heads);
 kvzip_status kvzip_select(const float* scores, int64_t N, int64_t k, int64_t n_heads,
                           uint8_t* keep, int64_t* offsets, float* threshold,
                           void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * kvzip_select given the round-1 histogram of the scores (score_hist, as
+ * kvzip_score_colmax_hist leaves it for a context's last chunk): the scores
+ * are read once instead of twice.  The kernel checks the histogram against
+ * the scores it reads (the counts above and inside the threshold's bin).  If
+ * they disagree, nothing is kept: keep is all 0, offsets all 0, threshold
+ * +inf, and the status word records it (kvzip_workspace_status returns
+ * KVZIP_ERR_INVALID_ARG).  Other arguments as kvzip_select.  The pages have
+ * no counterpart.
+ */
+kvzip_status kvzip_select_hist(const float* scores, int64_t N, int64_t k, int64_t n_heads,
+                               const unsigned int* score_hist, uint8_t* keep, int64_t* offsets,
+                               float* threshold, void* workspace, size_t ws_bytes,
+                               void* stream);
 
 /*
  * kvzip_select without a workspace, for callers that cannot allocate device

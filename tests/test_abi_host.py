@@ -125,6 +125,16 @@ def test_select_rejects_bad_arguments(kz):
     assert _select(kz, N=1 << 31, k=0, H=1) == kz.ERR_INVALID_ARG
 
 
+def test_histogram_entry_points_reject_a_missing_histogram(kz):
+    L = kz.library()
+    assert L.kvzip_select_hist(FAKE, 1000, 300, 10, None, FAKE, FAKE, None, FAKE, 1 << 30,
+                               None) == kz.ERR_INVALID_ARG
+    assert L.kvzip_select_hist(FAKE, 1000, 300, 10, FAKE + 2, FAKE, FAKE, None, FAKE, 1 << 30,
+                               None) == kz.ERR_INVALID_ARG        # 4-byte aligned counts
+    assert L.kvzip_score_colmax_hist(kz.BF16, FAKE, FAKE, FAKE, FAKE, 2, 4, 64, 100, 128, 0.0,
+                                     None, FAKE, 1 << 30, None) == kz.ERR_INVALID_ARG
+
+
 def _compact(kz, **over):
     a = dict(k=FAKE, v=FAKE, keep=FAKE, off=FAKE, H=4, n_c=100, d=128, ko=FAKE, vo=FAKE, pos=None,
              ws=FAKE, ws_bytes=1 << 30)
