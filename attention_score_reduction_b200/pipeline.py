@@ -72,21 +72,21 @@ class Compressor:
         self.offsets = torch.empty(units + 1, dtype=torch.int64, device=self.device)
         self.threshold = torch.empty(1, dtype=torch.float32, device=self.device)
         # round-1 histogram of the final scores, counted by the last chunk's
-        # column-max pass; the one-GPU selection then reads the scores once
-        self.score_hist = kz.new_score_hist(self.device) if group is None else None
+        # column-max pass: the one-GPU selection then reads the scores once, and
+        # a sharded selection skips its first histogram pass
+        self.score_hist = kz.new_score_hist(self.device)
         self.hist_ready = False
         self.launches = 0
 
     def reset(self):
         self.scores.zero_()
-        if self.score_hist is not None:
-            self.score_hist.zero_()
+        self.score_hist.zero_()
         self.hist_ready = False
 
     def score_chunk(self, q, k_ctx, k_self, scale: float = 0.0, stream=None, last: bool = False):
         """One chunk; ``last`` (the context's final chunk) also counts the
         final scores in the selection's round-1 histogram."""
-        if last and self.score_hist is not None:
+        if last:
             kz.score_chunk(q, k_ctx, k_self, self.scores, self.score_ws, scale, stream, "lse")
             self.launches += kz.last_launch_count()
             kz.score_chunk(q, k_ctx, k_self, self.scores, self.score_ws, scale, stream, "colmax",
@@ -114,10 +114,12 @@ class Compressor:
             return kept
         from . import sharded
         k = kz.keep_count(r, self.units_global * self.n_c)
+        given = self.score_hist if self.hist_ready else None
         sharded.select_sharded(self.scores, k, self.group, workspace=self.select_ws,
                                keep=self.keep, offsets=self.offsets, threshold=self.threshold,
-                               stream=stream)
-        self.launches += 13   # begin, 3 x (histogram, pick), tie count, five-kernel mask
+                               stream=stream, round1_hist=given)
+        # begin, 3 x (histogram, pick), tie count, five-kernel mask; one histogram fewer if given
+        self.launches += 13 if given is None else 12
         return self.keep_capacity(r)
 
     def compact(self, k_ctx, v, kept: int, k_out=None, v_out=None, pos_out=None, stream=None):

@@ -30,10 +30,14 @@ import torch.distributed as dist
 def select_sharded(scores_local: torch.Tensor, k: int, group=None, backend=None,
                    workspace: torch.Tensor | None = None, keep: torch.Tensor | None = None,
                    offsets: torch.Tensor | None = None, threshold: torch.Tensor | None = None,
-                   stream=None):
+                   stream=None, round1_hist: torch.Tensor | None = None):
     """Keep the k largest scores of the whole context (k is the GLOBAL count).
 
     scores_local: this rank's scores [n_heads_local][n_c] float32.
+    round1_hist: optionally, the round-1 histogram of exactly these scores
+    (SCORE_HIST_BINS counts, as the last chunk's kvzip_score_colmax_hist leaves
+    it); it replaces this rank's first histogram pass.  Like the histograms
+    the ranks exchange, it is trusted as given.
     Returns (keep uint8 [n_heads_local * n_c], offsets int64 [n_heads_local + 1]
     over this rank's heads, threshold float32 [1] = the k-th largest score of
     the whole context, +inf when k == 0).
@@ -57,8 +61,14 @@ def select_sharded(scores_local: torch.Tensor, k: int, group=None, backend=None,
 
     backend.shard_begin(k, workspace, stream)
     for r in range(3):
-        hist = torch.empty(backend.shard_bins(r), dtype=torch.int64, device=dev)
-        backend.shard_hist(flat, r, hist, workspace, stream)
+        if r == 0 and round1_hist is not None:
+            if round1_hist.numel() != backend.shard_bins(0):
+                raise ValueError("round1_hist must hold shard_bins(0) counts")
+            # a copy (also when it is int64 already): the all-reduce works in place
+            hist = round1_hist.to(torch.int64, copy=True)
+        else:
+            hist = torch.empty(backend.shard_bins(r), dtype=torch.int64, device=dev)
+            backend.shard_hist(flat, r, hist, workspace, stream)
         _all_reduce_sum(hist, group, on_host)
         backend.shard_pick(hist, r, threshold, workspace, stream)
     n_ties = torch.empty(1, dtype=torch.int64, device=dev)

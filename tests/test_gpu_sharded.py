@@ -31,8 +31,9 @@ def kz():
     return kvzip
 
 
-def _run_ranks(kz, parts, k):
-    """The shard protocol for several ranks in one process."""
+def _run_ranks(kz, parts, k, given=None):
+    """The shard protocol for several ranks in one process.  ``given``: per
+    rank, its round-1 histogram, used instead of its first histogram pass."""
     dev = parts[0].device
     wss = [kz.shard_workspace(p.numel(), p.shape[0], dev) for p in parts]
     thr = [torch.full((1,), -1.0, device=dev) for _ in parts]
@@ -40,7 +41,10 @@ def _run_ranks(kz, parts, k):
         kz.shard_begin(k, ws)
     for r in range(3):
         hists = []
-        for p, ws in zip(parts, wss):
+        for i, (p, ws) in enumerate(zip(parts, wss)):
+            if r == 0 and given is not None:
+                hists.append(given[i].to(torch.int64, copy=True))
+                continue
             h = torch.full((kz.shard_bins(r),), -5, dtype=torch.int64, device=dev)
             kz.shard_hist(p.reshape(-1), r, h, ws)
             hists.append(h)
@@ -95,6 +99,32 @@ def test_shard_protocol_matches_global_selection(kz, heads, n_c, levels):
             h0 += h
         if k:
             assert all(t == thr_ref for t in thr)
+
+
+def test_shard_protocol_with_round1_histograms_from_the_scorer(kz):
+    """Each rank's round-1 histogram counted by its last chunk's pass 2
+    (kvzip_score_colmax_hist) replaces its first histogram pass; the result is
+    still the global selection."""
+    g = torch.Generator().manual_seed(21)
+    B, G, n_in, n_c, d = 6, 4, 80, 900, 128
+    q = torch.randn(B, G, n_in, d, generator=g).to(torch.bfloat16).cuda()
+    k_ctx = torch.randn(B, n_c, d, generator=g).to(torch.bfloat16).cuda()
+    ks = torch.randn(B, n_in, d, generator=g).to(torch.bfloat16).cuda()
+    parts, given = [], []
+    for h0, h1 in ((0, 2), (2, 6)):   # two ranks, uneven
+        S = torch.zeros(h1 - h0, n_c, device="cuda")
+        hist = kz.new_score_hist()
+        kz.score_chunk(q[h0:h1].contiguous(), k_ctx[h0:h1].contiguous(), ks[h0:h1].contiguous(),
+                       S, hist=hist)
+        parts.append(S)
+        given.append(hist)
+    s_all = torch.cat([p.reshape(-1) for p in parts]).cpu().numpy()
+    for r in (0.3, 0.5):
+        k = oracle.keep_count(r, s_all.size)
+        out, thr = _run_ranks(kz, parts, k, given)
+        keep_ref, off_ref, thr_ref = oracle.select(s_all, k, B)
+        assert np.array_equal(np.concatenate([o[0].cpu().numpy() for o in out]), keep_ref)
+        assert all(t == thr_ref for t in thr)
 
 
 def test_shard_protocol_signed_zero(kz):

@@ -66,7 +66,7 @@ def test_score_flops_counts_pairs():
     assert f["pass1"] == 2 * 4 * 2 * (R * 7 + 3 * 5 * 6 // 2)
 
 
-def _shard_worker(rank, world, port, q, heads, n_c, levels, ks):
+def _shard_worker(rank, world, port, q, heads, n_c, levels, ks, given=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
@@ -75,23 +75,31 @@ def _shard_worker(rank, world, port, q, heads, n_c, levels, ks):
         s = synth.random_scores(sum(heads), n_c, seed=7 + levels, levels=levels)
         h0 = sum(heads[:rank])
         mine = s[h0:h0 + heads[rank]].contiguous()
+        hist = None
+        if given:   # this rank's round-1 histogram, as its last chunk's pass 2 would count it
+            import numpy as np
+            u = mine.reshape(-1).numpy().view(np.uint32)
+            hist = torch.from_numpy(np.bincount((u & 0x7FFFFFFF) >> 19, minlength=8192))
         out = []
         for k in ks:
-            keep, off, thr = sharded.select_sharded(mine, k, backend=shard_fake)
+            keep, off, thr = sharded.select_sharded(mine, k, backend=shard_fake, round1_hist=hist)
             out.append((keep.numpy().copy(), off.numpy().copy(), float(thr.item())))
         q.put((rank, out))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("heads,n_c,levels", [((3, 5), 300, 0), ((4, 4), 257, 8), ((2, 6), 100, 2),
-                                              ((5, 3), 64, 1)])
-def test_sharded_selection_exchange_matches_global(heads, n_c, levels):
+@pytest.mark.parametrize("heads,n_c,levels,given", [((3, 5), 300, 0, False), ((4, 4), 257, 8, False),
+                                                    ((2, 6), 100, 2, False), ((5, 3), 64, 1, False),
+                                                    ((3, 5), 300, 0, True), ((4, 4), 257, 8, True)])
+def test_sharded_selection_exchange_matches_global(heads, n_c, levels, given):
     """Two gloo ranks, each holding a run of heads (uneven splits), run the
     sharded selection's exchange (histogram all-reduce per radix round, tie
     count all-gather); the concatenated masks, the per-rank offsets and the
     threshold equal the oracle's global selection, including tie-heavy arrays
-    where the ties at the threshold straddle the two ranks."""
+    where the ties at the threshold straddle the two ranks.  With ``given``,
+    each rank passes its round-1 histogram instead of running the first
+    histogram pass."""
     import numpy as np
 
     import oracle
@@ -101,7 +109,8 @@ def test_sharded_selection_exchange_matches_global(heads, n_c, levels):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = 30500 + (os.getpid() % 1000) + 7 * levels
-    procs = [ctx.Process(target=_shard_worker, args=(r, 2, port, q, heads, n_c, levels, ks))
+    port += 3 if given else 0
+    procs = [ctx.Process(target=_shard_worker, args=(r, 2, port, q, heads, n_c, levels, ks, given))
              for r in range(2)]
     for p in procs:
         p.start()
