@@ -76,6 +76,7 @@ class Compressor:
         # a sharded selection skips its first histogram pass
         self.score_hist = kz.new_score_hist(self.device)
         self.hist_ready = False
+        self.unit_ws = {}   # (u0, u1) -> workspace of score_units
         self.launches = 0
 
     def reset(self):
@@ -86,14 +87,28 @@ class Compressor:
     def score_chunk(self, q, k_ctx, k_self, scale: float = 0.0, stream=None, last: bool = False):
         """One chunk; ``last`` (the context's final chunk) also counts the
         final scores in the selection's round-1 histogram."""
+        self._score(q, k_ctx, k_self, self.scores, self.score_ws, scale, stream, last)
+
+    def score_units(self, u0: int, u1: int, q, k_ctx, k_self, scale: float = 0.0, stream=None,
+                    last: bool = False):
+        """One chunk for units [u0, u1) only (q, k_ctx, k_self hold every unit),
+        with a workspace of its own for those units' row normalisers."""
+        ws = self.unit_ws.get((u0, u1))
+        if ws is None:
+            ws = self.unit_ws[(u0, u1)] = kz.new_score_workspace(u1 - u0, self.G, self.max_n_in,
+                                                                 self.device)
+        self._score(q[u0:u1], k_ctx[u0:u1], k_self[u0:u1], self.scores[u0:u1], ws, scale, stream,
+                    last)
+
+    def _score(self, q, k_ctx, k_self, scores, ws, scale, stream, last):
         if last:
-            kz.score_chunk(q, k_ctx, k_self, self.scores, self.score_ws, scale, stream, "lse")
+            kz.score_chunk(q, k_ctx, k_self, scores, ws, scale, stream, "lse")
             self.launches += kz.last_launch_count()
-            kz.score_chunk(q, k_ctx, k_self, self.scores, self.score_ws, scale, stream, "colmax",
+            kz.score_chunk(q, k_ctx, k_self, scores, ws, scale, stream, "colmax",
                            hist=self.score_hist)
             self.hist_ready = True
         else:
-            kz.score_chunk(q, k_ctx, k_self, self.scores, self.score_ws, scale, stream)
+            kz.score_chunk(q, k_ctx, k_self, scores, ws, scale, stream)
         self.launches += kz.last_launch_count()
 
     def keep_capacity(self, r: float) -> int:
@@ -146,9 +161,10 @@ class Compressor:
         return Compressed(k_out, v_out, pos, self.offsets, kept, self.threshold)
 
     def check_status(self, stream=None):
-        s = kz.workspace_status(self.score_ws, stream)
-        if s != kz.OK:
-            raise kz.KvzipError(s, "scoring kernels")
+        for ws in [self.score_ws] + list(self.unit_ws.values()):
+            s = kz.workspace_status(ws, stream)
+            if s != kz.OK:
+                raise kz.KvzipError(s, "scoring kernels")
         if self.group is None:
             s = kz.workspace_status(self.select_ws, stream)
             if s != kz.OK:
@@ -156,7 +172,8 @@ class Compressor:
 
 
 def compress_from_host(comp: Compressor, k_ctx_h, v_h, q_chunks_h, ks_chunks_h, r: float,
-                       dev_bufs: dict, host_out: dict | None = None, scale: float = 0.0):
+                       dev_bufs: dict, host_out: dict | None = None, scale: float = 0.0,
+                       key_slices: int = 4):
     """Upload host inputs, compress, and read the compacted cache back.
 
     k_ctx_h, v_h: pinned host [units][n_c][d]; q_chunks_h / ks_chunks_h: lists of
@@ -164,26 +181,43 @@ def compress_from_host(comp: Compressor, k_ctx_h, v_h, q_chunks_h, ks_chunks_h, 
     reusable device tensors: "k_ctx", "v", and lists "q", "ks" of chunk buffers.
     When the lists are shorter than the chunk list they are used as a ring:
     chunk c goes into buffer c % len, and its upload waits until the scorer has
-    finished the chunk that last used that buffer.  V is uploaded after the first
-    chunk's inputs, under the scoring; only compaction waits for it.  ``host_out`` (pinned)
-    receives "k", "v", "pos", "offsets".  Uploads run on a side stream, each
-    chunk's upload recorded by an event the scorer waits on.
+    finished the chunk that last used that buffer.  ``host_out`` (pinned)
+    receives "k", "v", "pos", "offsets".  Uploads run on a side stream in the
+    order the scorer needs them, each recorded by an event the scorer waits on:
+    the first chunk's inputs, then the context keys in ``key_slices`` runs of
+    units (the first chunk is scored run by run as its keys arrive), then each
+    later chunk's inputs followed by a piece of V, which only compaction needs.
     Returns (Compressed on the device, host_out, bytes_h2d, bytes_d2h).
     """
     main = torch.cuda.current_stream()
     copy = dev_bufs.setdefault("_copy_stream", torch.cuda.Stream())
     n_buf = len(dev_bufs["q"])
-    if n_buf == 0 or len(dev_bufs["ks"]) != n_buf or len(q_chunks_h) != len(ks_chunks_h):
+    n_chunks = len(q_chunks_h)
+    if n_buf == 0 or len(dev_bufs["ks"]) != n_buf or n_chunks != len(ks_chunks_h):
         raise ValueError("need matching lists of chunk inputs and device chunk buffers")
+    units = comp.units
+    n_sl = max(1, min(key_slices, units)) if n_chunks else 1
+    k_runs = [(units * i // n_sl, units * (i + 1) // n_sl) for i in range(n_sl)]
+    n_vp = max(1, min(units, n_chunks - 1))           # V pieces, one behind each later chunk
+    v_runs = [(units * i // n_vp, units * (i + 1) // n_vp) for i in range(n_vp)]
     copy.wait_stream(main)          # device buffers are free once earlier work is done
-    h2d = 0
-    with torch.cuda.stream(copy):
-        dev_bufs["k_ctx"].copy_(k_ctx_h, non_blocking=True)
-        h2d += k_ctx_h.numel() * k_ctx_h.element_size()
-        ev_k = torch.cuda.Event()
-        ev_k.record(copy)
     comp.reset()
-    main.wait_event(ev_k)           # scoring needs the keys; V only at compaction
+    h2d = 0
+    ev_v = []
+
+    def upload(dst, src_h):
+        nonlocal h2d
+        dst.copy_(src_h, non_blocking=True)
+        h2d += src_h.numel() * src_h.element_size()
+
+    def upload_v(p):
+        a, b = v_runs[p]
+        with torch.cuda.stream(copy):
+            upload(dev_bufs["v"][a:b], v_h[a:b])
+            ev = torch.cuda.Event()
+            ev.record(copy)
+        ev_v.append(ev)
+
     freed = [None] * n_buf          # event: the scorer is done with this ring slot
     for c, (qh, ksh) in enumerate(zip(q_chunks_h, ks_chunks_h)):
         slot = c % n_buf
@@ -194,29 +228,41 @@ def compress_from_host(comp: Compressor, k_ctx_h, v_h, q_chunks_h, ks_chunks_h, 
         with torch.cuda.stream(copy):
             if freed[slot] is not None:
                 copy.wait_event(freed[slot])
-            qd.copy_(qh, non_blocking=True)
-            ksd.copy_(ksh, non_blocking=True)
-            h2d += qh.numel() * qh.element_size() + ksh.numel() * ksh.element_size()
+            upload(qd, qh)
+            upload(ksd, ksh)
             up = torch.cuda.Event()
             up.record(copy)
-        main.wait_event(up)
-        comp.score_chunk(qd, dev_bufs["k_ctx"], ksd, scale, last=c == len(q_chunks_h) - 1)
+        last = c == n_chunks - 1
+        if c == 0:                  # the keys, run by run, each scored as it lands
+            ev_k = []
+            with torch.cuda.stream(copy):
+                for a, b in k_runs:
+                    upload(dev_bufs["k_ctx"][a:b], k_ctx_h[a:b])
+                    ev = torch.cuda.Event()
+                    ev.record(copy)
+                    ev_k.append(ev)
+            main.wait_event(up)
+            for (a, b), ev in zip(k_runs, ev_k):
+                main.wait_event(ev)
+                if n_sl == 1:
+                    comp.score_chunk(qd, dev_bufs["k_ctx"], ksd, scale, last=last)
+                else:
+                    comp.score_units(a, b, qd, dev_bufs["k_ctx"], ksd, scale, last=last)
+        else:
+            main.wait_event(up)
+            comp.score_chunk(qd, dev_bufs["k_ctx"], ksd, scale, last=last)
+            if c - 1 < n_vp:
+                upload_v(c - 1)
         done = torch.cuda.Event()
         done.record(main)
         freed[slot] = done
-        if c == 0:                  # V rides behind the first chunk, under the scoring
+    if n_chunks <= 1:
+        if not n_chunks:            # no chunks: the keys still go up for compaction
             with torch.cuda.stream(copy):
-                dev_bufs["v"].copy_(v_h, non_blocking=True)
-                h2d += v_h.numel() * v_h.element_size()
-                ev_v = torch.cuda.Event()
-                ev_v.record(copy)
-    if not q_chunks_h:
-        with torch.cuda.stream(copy):
-            dev_bufs["v"].copy_(v_h, non_blocking=True)
-            h2d += v_h.numel() * v_h.element_size()
-            ev_v = torch.cuda.Event()
-            ev_v.record(copy)
-    main.wait_event(ev_v)
+                upload(dev_bufs["k_ctx"], k_ctx_h)
+        upload_v(0)
+    for ev in ev_v:
+        main.wait_event(ev)
     kept = comp.select(r)
     if comp.group is not None:    # this rank's share of the global count (one small read)
         kept = int(comp.offsets[-1])
