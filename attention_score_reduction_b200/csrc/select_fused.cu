@@ -26,6 +26,12 @@
 //   F  every block sets the mask of its kept candidates; grid barrier.
 //   G  block 0 turns the per-head kept counts into offsets and writes tau.
 //
+// Given the round-1 histogram (kvzip_select_hist; the last chunk's pass 2
+// counts it while writing the final scores), A and its barrier are skipped and
+// the scores are read once.  After C every block checks the histogram against
+// what C counted (the candidates in b1 and the scores kept above it); on a
+// mismatch nothing is kept and the status word records it.
+//
 // Scores are ordered by the bits of |s| (mag): the value order for s >= 0,
 // with -0.0 equal to 0.0.
 //
