@@ -2,10 +2,11 @@
 
 A small multi-layer context with more chunks than device chunk buffers, so
 the uploads reuse a ring of two device slots (each upload waits until the
-scorer is done with the slot's previous chunk) and V arrives after the first
-chunk, under the scoring.  The packed cache, positions and offsets read back
-to the host must equal the device-resident path's (Compressor.compress) bit
-for bit, and the scores must too: same kernels, same order.
+scorer is done with the slot's previous chunk).  The context keys arrive in
+runs of units (1, 3 and 4 runs: the first chunk is scored run by run) and V
+in pieces behind the later chunks.  The packed cache, positions and offsets
+read back to the host must equal the device-resident path's
+(Compressor.compress) bit for bit, and the scores must too: same kernels.
 """
 import pytest
 import torch
@@ -17,7 +18,8 @@ def _pinned(t):
     return t.contiguous().pin_memory()
 
 
-def test_host_pipeline_matches_device_path_with_buffer_ring():
+@pytest.mark.parametrize("key_slices", [1, 3, 4])
+def test_host_pipeline_matches_device_path_with_buffer_ring(key_slices):
     from attention_score_reduction_b200 import build
     build.build()
     from attention_score_reduction_b200 import pipeline, synth
@@ -49,7 +51,7 @@ def test_host_pipeline_matches_device_path_with_buffer_ring():
     for _ in range(2):   # twice: the second pass reuses every buffer
         out, host_out, h2d, d2h = pipeline.compress_from_host(
             comp, _pinned(k_ctx), _pinned(v), [_pinned(q) for q, _ in chunks],
-            [_pinned(ks) for _, ks in chunks], 0.3, bufs, host_out)
+            [_pinned(ks) for _, ks in chunks], 0.3, bufs, host_out, key_slices=key_slices)
         torch.cuda.synchronize()
         comp.check_status()
         assert torch.equal(comp.scores, ref.scores)
@@ -62,3 +64,31 @@ def test_host_pipeline_matches_device_path_with_buffer_ring():
         sum(q.numel() * q.element_size() + ks.numel() * ks.element_size() for q, ks in chunks)
     assert h2d == in_bytes
     assert d2h == kept * wl.d * 2 * 2 + kept * 4 + (wl.units + 1) * 8
+
+
+def test_host_pipeline_single_chunk_context():
+    """One chunk: it is both the first chunk (scored run by run as the keys
+    land) and the last (its runs count the round-1 histogram); V goes up whole."""
+    from attention_score_reduction_b200 import build
+    build.build()
+    from attention_score_reduction_b200 import pipeline, synth
+    wl = synth.Workload("host_one", L=1, H=4, G=2, d=128, n_c=500, m=600, r=(0.3,),
+                        hi_frac=0.01, sinks=4, cfg_id=92)
+    assert wl.n_chunks == 1
+    dev = torch.device("cuda", 0)
+    k_ctx, v = synth.context_kv(wl)
+    q, ks = synth.chunk_qk(wl, 0)
+    ref = pipeline.Compressor(wl.units, wl.n_c, wl.d, wl.G, q.shape[2], device=dev)
+    out_ref = ref.compress(k_ctx.to(dev), v.to(dev), [(q.to(dev), ks.to(dev))], r=0.3)
+    comp = pipeline.Compressor(wl.units, wl.n_c, wl.d, wl.G, q.shape[2], device=dev)
+    bufs = {"k_ctx": torch.empty_like(k_ctx, device=dev), "v": torch.empty_like(v, device=dev),
+            "q": [torch.empty_like(q, device=dev)], "ks": [torch.empty_like(ks, device=dev)]}
+    out, _, h2d, _ = pipeline.compress_from_host(comp, _pinned(k_ctx), _pinned(v), [_pinned(q)],
+                                                 [_pinned(ks)], 0.3, bufs)
+    torch.cuda.synchronize()
+    comp.check_status()
+    assert torch.equal(comp.scores, ref.scores)
+    assert torch.equal(out.offsets, out_ref.offsets)
+    assert torch.equal(out.k.view(torch.int16), out_ref.k.view(torch.int16))
+    assert torch.equal(out.pos, out_ref.pos)
+    assert h2d == sum(t.numel() * t.element_size() for t in (k_ctx, v, q, ks))
