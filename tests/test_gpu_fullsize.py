@@ -66,19 +66,30 @@ def test_fullsize_scores_sampled_units(kz, full, chunk, units):
 
 def test_fullsize_select_and_compact(kz, full):
     """Global selection over 32 x 8 x 131072 scores (from the GPU's chunk-0
-    scores) is bit-exact at r = 0.3 and 0.5; compacted rows of sampled heads
-    equal their source rows."""
+    scores) is bit-exact at r = 0.3 and 0.5, read twice (kvzip_select) and
+    read once given the round-1 histogram that chunk 0's pass 2 counted
+    (kvzip_select_hist); compacted rows of sampled heads equal their source
+    rows."""
     from attention_score_reduction_b200 import synth
     wl, k_ctx, v = full
     q, ks = synth.chunk_qk(wl, 0, device=k_ctx.device)
     S = torch.zeros(wl.units, wl.n_c, device=k_ctx.device)
-    kz.score_chunk(q, k_ctx, ks, S)
+    hist = kz.new_score_hist(k_ctx.device)
+    kz.score_chunk(q, k_ctx, ks, S, hist=hist)
     del q, ks
     s_host = S.reshape(-1).cpu().numpy()
+    u = s_host.view(np.uint32)
+    assert np.array_equal(hist.cpu().numpy().astype(np.int64),
+                          np.bincount((u & 0x7FFFFFFF) >> 19, minlength=8192))
     for r in (0.3, 0.5):
         k = kz.keep_count(r, S.numel())
-        keep, off, thr = kz.select(S.reshape(-1), k, wl.units)
         keep_ref, off_ref, thr_ref = oracle.select(s_host, k, wl.units)
+        keep_h, off_h_given, thr_h = kz.select(S.reshape(-1), k, wl.units, hist=hist)
+        assert np.array_equal(off_h_given.cpu().numpy(), off_ref)
+        assert np.array_equal(keep_h.cpu().numpy(), keep_ref)
+        assert float(thr_h.item()) == thr_ref
+        del keep_h
+        keep, off, thr = kz.select(S.reshape(-1), k, wl.units)
         assert np.array_equal(off.cpu().numpy(), off_ref)
         assert np.array_equal(keep.cpu().numpy(), keep_ref)
         assert float(thr.item()) == thr_ref
