@@ -265,6 +265,28 @@ def pin_select_bruteforce(o):
 
 # ------------------------------------------------------------- compaction pins
 
+def pin_select_signed_zero_and_inf(o):
+    """Scores compare by value (the ordering reading): -0.0 equals 0.0, so the
+    zeros of both signs tie and go lowest index first, and +inf ranks above
+    every finite score.  Exhaustive search over all subsets of 8 scores whose
+    value codes are exact integers (-0.0 and 0.0 both code 0, +inf codes 9)."""
+    from itertools import combinations
+    s = np.array([0.0, -0.0, 0.5, np.inf, -0.0, 0.25, 0.0, np.inf], dtype=np.float32)
+    code = {0.0: 0, 0.25: 1, 0.5: 2}
+    c = [9 if np.isinf(x) else code[float(abs(x))] for x in s]
+    for k in range(0, 9):
+        best = None
+        for sub in combinations(range(8), k):
+            key = (sum(c[i] for i in sub), tuple(-i for i in sorted(sub)))
+            if best is None or key > best[0]:
+                best = (key, sub)
+        keep, off, thr = o.select(s, k, 2)
+        assert set(np.nonzero(keep)[0].tolist()) == set(best[1]), k
+        if k:
+            assert thr == min(s[list(best[1])])   # -0.0 == 0.0
+        assert off[-1] == k
+
+
 def pin_compact(o):
     """Compacted rows equal the source rows byte for byte; positions ascend in
     each head; kept bytes = k * d * 2 (bf16) * 2 (K and V)."""
@@ -466,7 +488,7 @@ def pin_expand_keep(o):
 
 SCORING_PINS = [pin_row_sums_and_range, pin_uniform_queries, pin_logistic, pin_dominant_key,
                 pin_bruteforce_unchunked, pin_invariants, pin_rows_see_own_prefix]
-SELECT_PINS = [pin_keep_count, pin_select_properties, pin_select_bruteforce]
+SELECT_PINS = [pin_keep_count, pin_select_properties, pin_select_bruteforce, pin_select_signed_zero_and_inf]
 COMPACT_PINS = [pin_compact, pin_kv_size_table]
 DECODE_PINS = [pin_decode_closed_forms, pin_decode_matches_dense_over_kept]
 VARIANT_PINS = [pin_sum_aggregation, pin_uniform_budgets, pin_head_scores, pin_token_scores,

@@ -218,13 +218,28 @@ def _mut_expand_offsets_by_n_c(m):
     m.expand_keep = expand
 
 
+def _mut_select_raw_bits(m):
+    # scores ranked by their raw float bits as unsigned integers: -0.0 (0x80000000)
+    # then outranks every score, and any negative value outranks +inf
+    orig = m.select
+
+    def select(scores, k, n_heads):
+        s = np.asarray(scores, dtype=np.float32).reshape(-1)
+        as_rank = s.view(np.uint32).astype(np.float64)
+        keep, off, _ = orig(as_rank, k, n_heads)
+        thr = float(s[np.nonzero(keep)[0]][np.argmin(as_rank[keep.astype(bool)])]) if k else math.inf
+        return keep, off, thr
+    m.select = select
+
+
 MUTANTS = [_mut_drop_diagonal, _mut_anticausal, _mut_row_order, _mut_no_self_in_normaliser,
            _mut_no_scale, _mut_mean, _mut_sum_over_chunks, _mut_transposed_keys,
            _mut_floor_count, _mut_tie_high_index, _mut_uniform_head_budget,
            _mut_positions_descending, _mut_decode_no_scale, _mut_decode_wrong_head,
            _mut_sum_without_self, _mut_per_head_tie_high, _mut_head_scores_wrong_axis,
            _mut_head_scores_heads_major, _mut_token_scores_layers_only,
-           _mut_token_scores_first_head, _mut_expand_repeat, _mut_expand_offsets_by_n_c]
+           _mut_token_scores_first_head, _mut_expand_repeat, _mut_expand_offsets_by_n_c,
+           _mut_select_raw_bits]
 
 
 @pytest.mark.parametrize("mutate", MUTANTS, ids=lambda f: f.__name__)
