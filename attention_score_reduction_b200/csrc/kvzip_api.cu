@@ -426,10 +426,12 @@ size_t kvzip_decode_workspace_size(int64_t n_heads, int G, int d) {
 }
 
 kvzip_status kvzip_decode_attention(const void* q, const void* k_packed, const void* v_packed,
-                                    const int64_t* offsets, int64_t n_heads, int G, int d,
-                                    float scale, float* out, void* workspace, size_t ws_bytes,
-                                    void* stream) {
+                                    int64_t n_rows, const int64_t* offsets, int64_t n_heads,
+                                    int G, int d, float scale, float* out, void* workspace,
+                                    size_t ws_bytes, void* stream) {
   if (n_heads <= 0 || n_heads > 65535 || G <= 0) return KVZIP_ERR_INVALID_ARG;
+  if (n_rows < 0 || n_rows > INT32_MAX) return KVZIP_ERR_INVALID_ARG;
+  if (n_rows > 0 && (k_packed == nullptr || v_packed == nullptr)) return KVZIP_ERR_INVALID_ARG;
   if (d != 128 && d != 256) return d > 0 ? KVZIP_ERR_UNSUPPORTED : KVZIP_ERR_INVALID_ARG;
   if (G != 1 && G != 2 && G != 4 && G != 5 && G != 8) return KVZIP_ERR_UNSUPPORTED;
   if (!q || !offsets || !out || !workspace) return KVZIP_ERR_INVALID_ARG;
@@ -443,6 +445,7 @@ kvzip_status kvzip_decode_attention(const void* q, const void* k_packed, const v
   a.q = q;
   a.k = k_packed;
   a.v = v_packed;
+  a.n_rows = n_rows;
   a.offsets = offsets;
   a.n_heads = n_heads;
   a.G = G;

@@ -110,6 +110,7 @@ struct DecodeArgs {
   const void* q;          // [n_heads][G][d] bf16
   const void* k;          // [total][d] bf16, packed head-major
   const void* v;
+  int64_t n_rows;         // rows of k and of v
   const int64_t* offsets; // [n_heads + 1]
   int64_t n_heads;
   int G, d;

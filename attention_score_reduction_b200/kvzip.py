@@ -70,7 +70,7 @@ def _load() -> ctypes.CDLL:
         "kvzip_select_per_head_workspace_size": (sz, [i64, i64]),
         "kvzip_select_per_head": (i32, [vp, i64, i64, i64, vp, vp, vp, sz, vp]),
         "kvzip_decode_workspace_size": (sz, [i64, i32, i32]),
-        "kvzip_decode_attention": (i32, [vp, vp, vp, vp, i64, i32, i32, f32, vp, vp, sz, vp]),
+        "kvzip_decode_attention": (i32, [vp, vp, vp, i64, vp, i64, i32, i32, f32, vp, vp, sz, vp]),
         "kvzip_last_launch_count": (i32, []),
         "kvzip_debug_checks": (i32, []),
         "kvzip_debug_bounds_status": (i32, []),
@@ -490,8 +490,11 @@ def decode_attention(q: torch.Tensor, k_packed: torch.Tensor, v_packed: torch.Te
                                 device=dev)
     kp = k_packed if k_packed.numel() else None
     vp = v_packed if v_packed.numel() else None
-    _check(_lib.kvzip_decode_attention(_ptr(q), _ptr(kp), _ptr(vp), _ptr(offsets), n_heads, G, d,
-                                       float(scale), _ptr(out), _ptr(workspace),
+    if k_packed.shape != v_packed.shape:
+        raise ValueError("k_packed and v_packed must have the same shape")
+    n_rows = k_packed.shape[0] if k_packed.numel() else 0
+    _check(_lib.kvzip_decode_attention(_ptr(q), _ptr(kp), _ptr(vp), n_rows, _ptr(offsets),
+                                       n_heads, G, d, float(scale), _ptr(out), _ptr(workspace),
                                        workspace.numel(), _stream(stream)),
            "kvzip_decode_attention")
     return out

@@ -361,15 +361,20 @@ size_t kvzip_decode_workspace_size(int64_t n_heads, int G, int d);
  * over head h's kept rows K_h = k_packed[offsets[h] : offsets[h+1]] (same for V).
  * A head with no kept rows gives zeros.
  *   q         [n_heads][G][d] bf16, 16-byte aligned.
- *   k_packed, v_packed  [offsets[n_heads]][d] bf16 (may be NULL only if nothing is kept).
+ *   k_packed, v_packed  [n_rows][d] bf16 each, 16-byte aligned (may be NULL only
+ *             if n_rows is 0).  The kernel reads them by TMA tiles bounded by
+ *             n_rows, so no read leaves the buffers whatever offsets holds.
+ *   n_rows    rows of k_packed and of v_packed, 0 .. 2^31 - 1; at least
+ *             offsets[n_heads] (a head whose range is not inside [0, n_rows)
+ *             reads nothing and gives zeros).
  *   offsets   [n_heads + 1] int64 (device).
  *   G         1, 2, 4, 5 or 8; d 128 or 256; scale <= 0 selects 1/sqrt(d).
  *   out       [n_heads][G][d] float32.
  */
 kvzip_status kvzip_decode_attention(const void* q, const void* k_packed, const void* v_packed,
-                                    const int64_t* offsets, int64_t n_heads, int G, int d,
-                                    float scale, float* out, void* workspace, size_t ws_bytes,
-                                    void* stream);
+                                    int64_t n_rows, const int64_t* offsets, int64_t n_heads,
+                                    int G, int d, float scale, float* out, void* workspace,
+                                    size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------ variants */
 
@@ -439,7 +444,8 @@ int kvzip_last_launch_count(void);
  * both selection paths, the scorer's normaliser tiles and score updates, the
  * decode row ranges) test every such index against its buffer first; a failed
  * test skips the access and sets a flag (no trap, no fault).  Normal builds
- * carry no checks. */
+ * carry no checks, except that decode attention always skips a head whose
+ * rows leave its n_rows (the debug build also sets the flag for it). */
 int kvzip_debug_checks(void);
 
 /* Synchronise the current device, then report whether any bounds check failed

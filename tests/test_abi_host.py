@@ -165,19 +165,22 @@ def test_head_scores_rejects_bad_arguments(kz):
 def test_decode_rejects_bad_arguments(kz):
     lib = kz.library()
     f = lib.kvzip_decode_attention
-    ok = dict(q=FAKE, k=FAKE, v=FAKE, off=FAKE, H=8, G=4, d=128, scale=0.0, out=FAKE, ws=FAKE,
-              wsb=1 << 30)
+    ok = dict(q=FAKE, k=FAKE, v=FAKE, rows=1000, off=FAKE, H=8, G=4, d=128, scale=0.0, out=FAKE,
+              ws=FAKE, wsb=1 << 30)
 
     def call(**over):
         a = dict(ok)
         a.update(over)
-        return f(a["q"], a["k"], a["v"], a["off"], a["H"], a["G"], a["d"], a["scale"], a["out"],
-                 a["ws"], a["wsb"], None)
+        return f(a["q"], a["k"], a["v"], a["rows"], a["off"], a["H"], a["G"], a["d"], a["scale"],
+                 a["out"], a["ws"], a["wsb"], None)
     assert call(G=3) == kz.ERR_UNSUPPORTED
     assert call(d=64) == kz.ERR_UNSUPPORTED
     assert call(H=0) == kz.ERR_INVALID_ARG
     assert call(q=None) == kz.ERR_INVALID_ARG
     assert call(k=None) == kz.ERR_INVALID_ARG           # k without v
+    assert call(k=None, v=None) == kz.ERR_INVALID_ARG   # rows without buffers
+    assert call(rows=-1) == kz.ERR_INVALID_ARG
+    assert call(rows=1 << 31) == kz.ERR_INVALID_ARG
     assert call(q=FAKE + 8) == kz.ERR_INVALID_ARG
     assert call(wsb=16) == kz.ERR_INVALID_ARG
     assert kz.decode_workspace_size(8, 4, 128) > 0

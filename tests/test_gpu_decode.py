@@ -76,3 +76,28 @@ def test_decode_long_heads(kz):
     """LLaMA3.1-8B layer shape at r = 0.3 of 16K keys: about 4900 kept rows per head."""
     q, ko, vo, off = _case(11, n_heads=8, n_c=16384, d=128, G=4, r=0.3)
     _check(kz, q, ko, vo, off)
+
+
+def test_decode_head_range_outside_the_buffer_reads_nothing(kz):
+    """offsets whose last head runs past the packed rows (n_rows, taken from
+    the tensors' shape): that head gives zeros and reads no row, the others
+    are exact.  The debug build also records the failed range check."""
+    q, ko, vo, off = _case(13, n_heads=4, n_c=900, d=128, G=4, r=0.3)
+    want = oracle.decode_attention(q.double().numpy(), ko.double().numpy(), vo.double().numpy(), off)
+    bad = off.copy()
+    bad[-1] = off[-1] + 40
+    got = kz.decode_attention(q.cuda(), ko.cuda(), vo.cuda(), torch.from_numpy(bad).cuda())
+    got = got.cpu().double().numpy()
+    assert np.allclose(got[:3], want[:3], rtol=1e-4, atol=1e-4)
+    assert not np.any(got[3])
+    lib = kz.library()
+    if lib.kvzip_debug_checks() == 1:
+        assert lib.kvzip_debug_bounds_status() == kz.ERR_BOUNDS   # reads and clears the flag
+
+
+def test_decode_buffer_with_spare_rows(kz):
+    """A packed buffer longer than offsets[n_heads] (spare rows after the last
+    head, as when it was sized for a larger budget): same result."""
+    q, ko, vo, off = _case(17, n_heads=3, n_c=1200, d=256, G=2, r=0.4)
+    pad = torch.randn(77, 256).to(torch.bfloat16)
+    _check(kz, q, torch.cat([ko, pad]), torch.cat([vo, pad]), off)
