@@ -229,3 +229,16 @@ def test_score_lse_layout(kz):
     assert lib.kvzip_score_lse_layout(4, 10, None, ctypes.byref(s)) == kz.ERR_INVALID_ARG
     assert lib.kvzip_score_lse_layout(1 << 20, 1 << 20, ctypes.byref(o),
                                       ctypes.byref(s)) == kz.ERR_UNSUPPORTED
+
+
+def test_c_caller_builds_against_header_and_library(tmp_path):
+    """The torch-free C caller (tests/c_abi_host_staging.c, run on a GPU by
+    test_gpu_c_abi_host.py) compiles with -Wall -Werror against include/kvzip.h
+    and links against libkvzip.so and the CUDA runtime."""
+    import shutil
+    if not (shutil.which("gcc") or shutil.which("cc")):
+        pytest.skip("no C compiler")
+    from tests.test_gpu_c_abi_host import _compile
+    exe = str(tmp_path / "c_abi_host_staging")
+    _compile(exe)
+    assert os.path.exists(exe)
