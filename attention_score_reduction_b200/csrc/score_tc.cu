@@ -37,6 +37,11 @@
 //                 accumulator in CH-column TMEM loads, so the tile's B tiles
 //                 alternate between two groups (four epilogue warps per
 //                 scheduler: the epilogue math is latency-bound with two).
+// Work items are (unit, 256-row block of A).  Pass 2 with A in shared memory
+// runs one persistent CTA per SM over the items: the B ring and the barrier
+// phases run on from item to item, the next item's A tiles are prefetched into
+// L2 and loaded once the issuers release the current ones.  Elsewhere each CTA
+// takes one item.
 // TMEM map (512 columns): the A tiles when they live there (D/2 columns each),
 // then the (tile, buffer) accumulators.
 // Every wait is bounded; on timeout the CTA records KVZIP_ERR_TIMEOUT in the
